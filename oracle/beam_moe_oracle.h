@@ -1,0 +1,90 @@
+/*
+ * beam_moe_oracle.h - plain, slow, fp64 CPU oracle of the Beam MoE block
+ * forward. TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the
+ * benchmark's CPU-baseline leg use it; the product path never does.
+ *
+ * What it computes is the block as the Hugging Face launch post "Welcome Beam"
+ * describes it (sections "Mixture of Experts" and "Residual Stream"), restated
+ * in the Russian-language summary (section "Экспертные блоки Mixture of
+ * Experts") and the Miles "Beam 1.0" recipe page (section 1, "Key
+ * highlights"): sigmoid scores over all experts, experts split into groups,
+ * the groups ranked by the sum of their two best scores, the best groups
+ * kept, the top experts taken inside them, SwiGLU experts, and a combine with
+ * normalized router weights scaled by the routed scale. It shares no code with
+ * the GPU library.
+ *
+ * Readings where the pages are silent (each is also listed in the design
+ * notes of the repository):
+ *  - ties break to the lower index, for groups and for experts;
+ *  - the selected ids are listed by descending score;
+ *  - "normalized router weights" means w_k = S * s_k / sum_j s_j over the
+ *    selected experts (renormalize = 1); renormalize = 0 gives S * s_k;
+ *  - bias_mode 0 adds the per-expert bias to the logits before the sigmoid;
+ *    bias_mode 1 adds it to the scores for choosing only (weights from the
+ *    unbiased scores), as in DeepSeek-V3, whose scheme the router follows;
+ *  - no intermediate rounding: everything is fp64 after exact conversion of
+ *    the bf16 / fp32 inputs.
+ *
+ * Arrays are row-major. bf16 values are passed as their 16-bit patterns.
+ * Functions return 0 on success and a negative code on a bad argument.
+ */
+#ifndef BEAM_MOE_ORACLE_H
+#define BEAM_MOE_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct {
+  int32_t hidden;      /* H */
+  int32_t inter;       /* I */
+  int32_t n_experts;   /* E */
+  int32_t n_group;     /* G, groups of E/G experts */
+  int32_t topk_group;  /* Gk kept groups */
+  int32_t top_k;       /* K experts per token */
+  int32_t renormalize; /* 1: weights normalized over the K selected */
+  int32_t bias_mode;   /* 0: bias on logits; 1: bias on choice only */
+  double routed_scale; /* S */
+} oracle_cfg;
+
+/*
+ * Routing of T tokens.
+ *   x        [T][H] bf16 bits;  w_router [E][H] fp32;  bias [E] fp32 or NULL.
+ * Outputs (any may be NULL):
+ *   ids      [T][K]  selected experts, descending choice score
+ *   weights  [T][K]  combine weights, routed scale included
+ *   scores   [T][K]  sigmoid score of each selected expert
+ *   kept     [T][Gk] kept groups, in the order they were chosen
+ *   margins  [T][2]  (group margin, expert margin): the gap between the last
+ *                    chosen and the best unchosen candidate, +inf if none
+ *   all_s    [T][E]  every expert's sigmoid score
+ */
+int oracle_route(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const float* w_router,
+                 const float* bias, int32_t* ids, double* weights, double* scores, int32_t* kept,
+                 double* margins, double* all_s);
+
+/*
+ * One SwiGLU expert on one token (x in fp64, length H):
+ *   g = Wg x, u = Wu x, a = silu(g) * u, y = Wd a       (y length H)
+ * w13 [2I][H] (rows 0..I-1 gate, I..2I-1 up), w2 [H][I], bf16 bits.
+ */
+int oracle_swiglu_expert(int32_t H, int32_t I, const double* x, const uint16_t* w13,
+                         const uint16_t* w2, double* y);
+
+/*
+ * Expert path and combine for T tokens given their routes:
+ *   out[t] = sum_k weights[t][k] * expert_{ids[t][k]}(x[t])     (fp64 [T][H])
+ * w13[e] / w2[e] point to expert e's weights; an expert no token selects may
+ * be NULL (a selected NULL expert is an error).
+ */
+int oracle_experts(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const int32_t* ids,
+                   const double* weights, const uint16_t* const* w13, const uint16_t* const* w2,
+                   double* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BEAM_MOE_ORACLE_H */
