@@ -1,0 +1,380 @@
+"""Benchmark of the Beam MoE block forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+A step is one whole block forward (router GEMM, top-k, scan, permute, gate/up
+grouped GEMM, down grouped GEMM, combine) over one batch of T synthetic tokens
+with Beam's shapes: hidden 5120, 256 SwiGLU experts of intermediate 2560 in 8
+groups of 32, top-4 groups, top-8 experts, routed scale 2.5. The default
+workload is decode (T = 64), the configuration the throughput is quoted on.
+Weights and inputs are synthetic and seeded (bf16 experts N(0, 0.02), fp32
+router N(0, 1/sqrt(5120)), bf16 activations N(0, 1)); they are resident in HBM
+before timing starts. The L2 cache is flushed (256 MB write) before every
+timed step, outside the timed interval. Timing: CUDA events on the launching
+stream around each step, summed over K steps, max over ranks.
+
+With N GPUs (torchrun, one process per GPU) every rank holds all experts and
+runs its own batch of T tokens: the block is data-parallel over tokens with
+no exchange, so scaling is weak and the only collective is the max of the
+timings.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this
+repository) on a bounded sample of the same workload on the host cores.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+
+import synth
+
+METRIC = "MoE-block tokens/s; achieved TFLOP/s or HBM GB/s as % of B200 roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+STAGES = ("router_gemm", "router_topk", "scan", "permute", "gateup_gemm", "down_gemm", "combine")
+KERNELS_PER_STEP = 7
+
+
+def describe(wl):
+    extra = ""
+    if wl.n_hot:
+        extra = f", router bias +{wl.hot_bias} on {wl.n_hot} experts"
+    if wl.n_centres:
+        extra = f", clustered inputs ({wl.n_centres} centres + N(0,{wl.sigma_x}) noise)"
+    return (f"Beam MoE block {wl.name}: T={wl.T}, hidden {wl.H}, {wl.E} SwiGLU experts of "
+            f"intermediate {wl.I} in {wl.G} groups of {wl.E // wl.G}, top-{wl.Gk} groups, "
+            f"top-{wl.K} experts, scale {wl.scale}{extra}")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic(wl, counts):
+    """Algorithmic work of one forward with these routed counts.
+
+    FLOPs: 6 H I per assignment (tensor cores) + 2 H E per token (FP32 router).
+    Bytes: 3 H I x 2 per touched expert, router weights, x and out.
+    gate/up kernel bytes: 2 I H x 2 per touched expert + permuted rows in + h out.
+    """
+    touched = int(np.count_nonzero(counts))
+    A = wl.T * wl.K
+    return {
+        "touched_experts": touched,
+        "expert_flops": 6.0 * wl.H * wl.I * A,
+        "router_flops": 2.0 * wl.H * wl.E * wl.T,
+        "block_bytes": touched * 3.0 * wl.H * wl.I * 2 + wl.E * wl.H * 4 + 2 * wl.T * wl.H * 2,
+        "gateup_bytes": touched * 2.0 * wl.I * wl.H * 2 + A * wl.H * 2 + A * wl.I * 2,
+        "gateup_flops": 4.0 * wl.H * wl.I * A,
+    }
+
+
+class ClockSampler:
+    """nvidia-smi samples of clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.out,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ reference arm
+
+class OracleSample:
+    """The fp64 CPU oracle (routing, experts and combine) on n sampled tokens of
+    a workload. The expert weights of the sampled tokens are generated once,
+    before any timed call."""
+
+    def __init__(self, wl, n_tokens, seed=synth.SEED):
+        import oracle
+
+        self.oracle = oracle
+        self.cfg = oracle.cfg_for(wl)
+        tokens = synth.sample_tokens(wl.T, n_tokens, seed)
+        self.n = len(tokens)
+        self.x = synth.host_x(wl, seed=seed)[tokens]
+        self.wr = synth.host_router(wl, seed)
+        self.b = synth.host_bias(wl, seed)
+        ids = oracle.route(self.cfg, self.x, self.wr, self.b)["ids"]
+        self.w13 = {int(e): synth.host_expert_w13(wl, int(e), seed) for e in np.unique(ids)}
+        self.w2 = {int(e): synth.host_expert_w2(wl, int(e), seed) for e in np.unique(ids)}
+        self.threads = min(self.n, int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)))
+        self.desc = (f"{self.n} of the {wl.T} tokens (seeded sample): full routing and all "
+                     f"{wl.K} experts per token in fp64; expert weights generated before timing")
+
+    def run(self):
+        """Returns (tokens/s, seconds) of one timed oracle pass over the sample."""
+        t0 = time.perf_counter()
+        r = self.oracle.route(self.cfg, self.x, self.wr, self.b)
+        self.oracle.experts(self.cfg, self.x, r["ids"], r["weights"], self.w13, self.w2)
+        dt = time.perf_counter() - t0
+        return self.n / dt, dt
+
+
+def oracle_sample_size(wl):
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return max(1, min(wl.T, cores, 16))
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    sample = OracleSample(wl, oracle_sample_size(wl))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, dt = sample.run()
+        if i >= args.warmup:
+            vals.append((v, dt))
+    value = sample.n * len(vals) / sum(dt for _, dt in vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * statistics.mean(dt for _, dt in vals),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": describe(wl), "T": wl.T, "sample_tokens_per_step": sample.n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": sample.threads,
+                         "kind": "oracle", "sample": sample.desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------------------- ours
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_moe_layer_beam_b200 as bm
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    stream = torch.cuda.current_stream()
+    st = stream.cuda_stream
+
+    cfg = bm.beam_cfg(wl.H, wl.I, wl.E, wl.G, wl.Gk, wl.K, wl.renormalize, 0, wl.scale)
+    # all ranks hold the same experts (seed 0); each rank routes its own tokens
+    w13 = torch.empty(wl.w13_elems, dtype=torch.int16, device=dev)
+    w2 = torch.empty(wl.w2_elems, dtype=torch.int16, device=dev)
+    synth.dev_w13(wl, w13.data_ptr(), st)
+    synth.dev_w2(wl, w2.data_ptr(), st)
+    wr = torch.from_numpy(synth.host_router(wl)).to(dev)
+    bias = synth.host_bias(wl)
+    b = None if bias is None else torch.from_numpy(bias).to(dev)
+    x = torch.empty((wl.T, wl.H), dtype=torch.int16, device=dev)
+    synth.dev_x(wl, x.data_ptr(), st, seed=synth.SEED + rank)
+    out = torch.empty((wl.T, wl.H), dtype=torch.int16, device=dev)
+    counts = torch.zeros(wl.E, dtype=torch.int32, device=dev)
+    ws = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    def step(trace=None):
+        if trace is None:
+            bm.beam_moe_forward(cfg, x, wr, b, w13, w2, out, ws, expert_counts=counts,
+                                stream=st)
+        else:
+            bm.beam_moe_forward_traced(cfg, x, wr, b, w13, w2, out, ws, trace,
+                                       expert_counts=counts, stream=st)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    flags = bm.beam_moe_check(ws, st)
+    if flags:
+        raise SystemExit(f"device status flags {flags:#x} after warm-up")
+
+    trace = bm.Trace(args.steps)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step(trace)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = sum(a.elapsed_time(c) for a, c in ev)
+    stage_ms = np.array(trace.read())  # [steps][stages]
+    flags = bm.beam_moe_check(ws, st)
+    if flags:
+        raise SystemExit(f"device status flags {flags:#x} in the timed region")
+
+    # end to end through the public call with host buffers: pinned x in, out back
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty_like(out, device="cpu").pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        j = i - args.warmup
+        if j >= 0:
+            e2e_ev[j][0].record(stream)
+        x.copy_(x_host, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+        if j >= 0:
+            e2e_ev[j][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(c) for a, c in e2e_ev)
+
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    ms_step = total_ms / args.steps
+    tokens = wl.T * world
+    value = tokens / (ms_step / 1000.0)
+    e2e_value = tokens / (e2e_ms / args.steps / 1000.0)
+
+    alg = algorithmic(wl, counts.cpu().numpy())
+    peaks, peak_kind = load_peaks()
+    gate_ms = float(stage_ms[:, 4].mean())
+    stage_mean = {n: float(stage_ms[:, i].mean()) for i, n in enumerate(STAGES)}
+    # the gate/up grouped GEMM dominates every configuration; its bound follows
+    # from its arithmetic intensity (flop per weight byte = rows per expert)
+    t_hbm = alg["gateup_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = alg["gateup_flops"] / (peaks["bf16_tflops"] * 1e12)
+    if t_hbm >= t_tc:
+        achieved = alg["gateup_bytes"] / (gate_ms / 1000.0) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = alg["gateup_flops"] / (gate_ms / 1000.0) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = "gateup_grouped_gemm"
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
+        else "fallback"
+    block_s = ms_step / 1000.0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(wl), "T": wl.T, "tokens_per_rank": wl.T,
+                   "l2": "flushed before every timed step (256 MB write, outside the events)",
+                   "parallelism": f"replicas x{world} (token data parallel, no exchange)"},
+        "roofline": roof,
+        "block": {"hbm_gbs": alg["block_bytes"] / block_s / 1e9,
+                  "hbm_frac": alg["block_bytes"] / block_s / 1e9 / peaks["hbm_gbs"],
+                  "tflops": alg["expert_flops"] / block_s / 1e12,
+                  "tensor_frac": alg["expert_flops"] / block_s / 1e12 / peaks["bf16_tflops"],
+                  "touched_experts": alg["touched_experts"]},
+        "stages_ms": stage_mean,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * wl.H * 2,
+                "d2h_bytes_per_step": wl.T * wl.H * 2},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = OracleSample(wl, oracle_sample_size(wl))
+        v, dt = sample.run()
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": sample.threads,
+                                "kind": "oracle", "sample": sample.desc, "seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    trace.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    wl = synth.workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

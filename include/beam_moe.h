@@ -1,0 +1,173 @@
+/*
+ * beam_moe.h - C ABI of the B200 (sm_100a) Beam MoE block forward.
+ *
+ * The operation is the routed-expert block of the Beam model as the Hugging
+ * Face launch post "Welcome Beam" describes it in section "Mixture of
+ * Experts": every expert is scored with a sigmoid of the router logits, the
+ * experts are split into n_group groups, the topk_group groups with the best
+ * sum of their two top scores are kept, the top_k experts inside them are
+ * chosen, each chosen expert is a SwiGLU MLP, and the expert outputs are
+ * combined with normalized router weights scaled by routed_scale (2.5 in
+ * Beam). Section "Residual Stream" of the same post fixes the router and the
+ * SwiGLU product to FP32; this library computes the router logits, the
+ * sigmoid, the selection, the weights and the SwiGLU product in FP32, the
+ * expert matmuls as BF16 x BF16 with FP32 accumulation.
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers named as device buffers must be device memory of the current
+ *    device; the caller owns all of them and the library never frees them.
+ *    All row-major. bf16 is passed as its 16-bit pattern (uint16_t).
+ *  - Every pointer must be 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ *    default stream); nothing synchronizes except beam_moe_check and
+ *    beam_moe_trace_read.
+ *  - Host-side checks run before any launch; on any error nothing is
+ *    launched and the outputs are untouched.
+ *  - T = 0 is a no-op that returns BEAM_MOE_OK.
+ *  - Results are bitwise reproducible run to run (no atomics on data).
+ *  - The library allocates no device memory: scratch lives in the caller's
+ *    workspace `ws` (size from beam_moe_workspace_size). A workspace must not
+ *    be shared by calls that may run concurrently.
+ */
+#ifndef BEAM_MOE_H
+#define BEAM_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BEAM_MOE_API __attribute__((visibility("default")))
+#else
+#define BEAM_MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Block configuration. Beam: {5120, 2560, 256, 8, 4, 8, 1, 0, 2.5f}.
+ * Supported: hidden and inter multiples of 128; n_experts <= 512 and a
+ * multiple of n_group; group size (n_experts / n_group) >= 2; top_k <= 32 and
+ * top_k <= topk_group * group size; see beam_moe_status for the codes. */
+typedef struct beam_moe_cfg {
+  int32_t hidden;      /* H: model width                                   */
+  int32_t inter;       /* I: expert intermediate width                     */
+  int32_t n_experts;   /* E: routed experts                                */
+  int32_t n_group;     /* G: expert groups (E / G experts each)            */
+  int32_t topk_group;  /* Gk: groups kept per token                        */
+  int32_t top_k;       /* K: experts per token                             */
+  int32_t renormalize; /* 1: w_k = S s_k / sum_j s_j; 0: w_k = S s_k       */
+  int32_t bias_mode;   /* 0: bias added to the logits before the sigmoid;
+                          1: bias added to the scores for choosing only,
+                             weights from the unbiased scores (DeepSeek-V3) */
+  float routed_scale;  /* S: multiplies the combined output (2.5 in Beam)  */
+} beam_moe_cfg;
+
+typedef enum beam_moe_status {
+  BEAM_MOE_OK = 0,
+  BEAM_MOE_ERR_INVALID_ARG = 1,       /* NULL / negative / inconsistent argument   */
+  BEAM_MOE_ERR_UNSUPPORTED_SHAPE = 2, /* configuration outside the supported set  */
+  BEAM_MOE_ERR_ALIGNMENT = 3,         /* a pointer is not 16-byte aligned         */
+  BEAM_MOE_ERR_WORKSPACE_TOO_SMALL = 4,
+  BEAM_MOE_ERR_CUDA = 5,              /* a CUDA runtime/driver call failed        */
+  BEAM_MOE_ERR_DEVICE_TIMEOUT = 6     /* a kernel gave up a bounded wait          */
+} beam_moe_status;
+
+typedef enum beam_moe_op {
+  BEAM_MOE_OP_ROUTE = 0,   /* beam_moe_route                            */
+  BEAM_MOE_OP_FORWARD = 1, /* beam_moe_forward, beam_moe_forward_routed */
+} beam_moe_op;
+
+/* Bytes of workspace the operation needs for T tokens (a pure host function). */
+BEAM_MOE_API beam_moe_status beam_moe_workspace_size(const beam_moe_cfg* cfg, int64_t T, beam_moe_op op,
+                                        size_t* bytes);
+
+/*
+ * Router and selection ("Welcome Beam", section "Mixture of Experts": sigmoid
+ * scores, groups ranked by the sum of their top two scores, top experts inside
+ * the kept groups, normalized weights).
+ *   x          [T][H] bf16, device            token activations
+ *   w_router   [E][H] fp32, device            router weights
+ *   bias       [E] fp32, device, or NULL      per-expert bias (see bias_mode)
+ *   topk_ids   [T][K] int32, device (out)     chosen experts, by descending
+ *                                             choice score, ties to lower id
+ *   topk_w     [T][K] fp32, device (out)      combine weights, S included
+ *   expert_counts [E] int32, device, or NULL (out): tokens routed to each expert
+ *   ws, ws_bytes  device workspace of at least
+ *                 beam_moe_workspace_size(cfg, T, BEAM_MOE_OP_ROUTE) bytes
+ */
+BEAM_MOE_API beam_moe_status beam_moe_route(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                               const float* w_router, const float* bias, int32_t* topk_ids,
+                               float* topk_w, int32_t* expert_counts, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/*
+ * Whole block forward: routing as beam_moe_route, then for every token
+ *   out[t] = sum_k topk_w[t][k] * Wd_e (silu(Wg_e x_t) * (Wu_e x_t)),  e = topk_ids[t][k]
+ * ("Welcome Beam", section "Mixture of Experts": SwiGLU experts of
+ * intermediate size I, outputs combined with normalized weights and scaled).
+ *   w13  [E][2I][H] bf16, device   rows 0..I-1 gate (Wg), rows I..2I-1 up (Wu)
+ *   w2   [E][H][I]  bf16, device   down projection (Wd)
+ *   out  [T][H]     bf16, device (out)
+ *   topk_ids, topk_w, expert_counts: optional device outputs (NULL to skip)
+ *   ws, ws_bytes: at least beam_moe_workspace_size(cfg, T, BEAM_MOE_OP_FORWARD)
+ */
+BEAM_MOE_API beam_moe_status beam_moe_forward(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                                 const float* w_router, const float* bias, const uint16_t* w13,
+                                 const uint16_t* w2, uint16_t* out, int32_t* topk_ids,
+                                 float* topk_w, int32_t* expert_counts, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/*
+ * Expert path with caller-supplied routes (routing replay, as the Miles
+ * "Beam 1.0" page's rollout routing replay option reuses recorded routes):
+ * the same as beam_moe_forward after its routing step.
+ *   topk_ids [T][K] int32, device: distinct experts per token, each in [0, E)
+ *   topk_w   [T][K] fp32, device: combine weights (any scale already applied)
+ * Ids are not re-validated on the device beyond a bounds check that flags
+ * BEAM_MOE_ERR_DEVICE_TIMEOUT-class status bit 0x100 in beam_moe_check.
+ */
+BEAM_MOE_API beam_moe_status beam_moe_forward_routed(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                                        const int32_t* topk_ids, const float* topk_w,
+                                        const uint16_t* w13, const uint16_t* w2, uint16_t* out,
+                                        int32_t* expert_counts, void* ws, size_t ws_bytes,
+                                        void* stream);
+
+/*
+ * Stage timing. A trace records CUDA events around each stage of the calls
+ * it is passed to: slot i of stage s is the time of that stage in the i-th
+ * traced call since the last reset. Stages: 0 router GEMM, 1 top-k and
+ * chunk counts, 2 scan, 3 permute, 4 gate/up grouped GEMM, 5 down grouped
+ * GEMM, 6 combine. beam_moe_trace_read synchronizes the recorded events.
+ */
+#define BEAM_MOE_N_STAGES 7
+typedef struct beam_moe_trace beam_moe_trace;
+BEAM_MOE_API beam_moe_status beam_moe_trace_create(int32_t capacity, beam_moe_trace** out);
+BEAM_MOE_API beam_moe_status beam_moe_trace_destroy(beam_moe_trace* trace);
+BEAM_MOE_API beam_moe_status beam_moe_trace_reset(beam_moe_trace* trace);
+/* ms[i * BEAM_MOE_N_STAGES + s] for i < *n_calls (at most capacity). */
+BEAM_MOE_API beam_moe_status beam_moe_trace_read(beam_moe_trace* trace, float* ms, int32_t* n_calls);
+BEAM_MOE_API beam_moe_status beam_moe_forward_traced(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                                        const float* w_router, const float* bias,
+                                        const uint16_t* w13, const uint16_t* w2, uint16_t* out,
+                                        int32_t* topk_ids, float* topk_w,
+                                        int32_t* expert_counts, void* ws, size_t ws_bytes,
+                                        void* stream, beam_moe_trace* trace);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device status word in the
+ * workspace. *device_flags (may be NULL) receives the raw bits: 0x1 producer,
+ * 0x2 MMA issuer, 0x4 epilogue gave up a bounded wait; 0x100 an expert id
+ * outside [0, E) reached the dispatch. Returns BEAM_MOE_ERR_DEVICE_TIMEOUT
+ * if any bit was set, BEAM_MOE_ERR_CUDA if the stream reports an error.
+ */
+BEAM_MOE_API beam_moe_status beam_moe_check(void* ws, size_t ws_bytes, void* stream, uint32_t* device_flags);
+
+/* Static description of a status code. */
+BEAM_MOE_API const char* beam_moe_status_string(beam_moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BEAM_MOE_H */

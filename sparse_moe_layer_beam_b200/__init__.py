@@ -1,0 +1,187 @@
+"""Beam MoE block forward on B200 (sm_100a): Python binding of libbeam_moe.so.
+
+Argument marshalling only: every step of the block runs in the library's CUDA
+kernels. Functions take torch tensors for device buffers (torch provides
+device memory and the current stream) and raise BeamMoeError on any non-OK
+status. There is no fallback: if the library is missing, the first call
+raises ImportError.
+
+The entry points mirror include/beam_moe.h one to one:
+beam_moe_workspace_size, beam_moe_route, beam_moe_forward,
+beam_moe_forward_routed, beam_moe_forward_traced, beam_moe_check, and the
+Trace wrapper of beam_moe_trace_*.
+"""
+import ctypes
+import os
+
+__all__ = ["BeamMoeCfg", "BeamMoeError", "Trace", "OP_ROUTE", "OP_FORWARD", "N_STAGES",
+           "STAGE_NAMES", "lib", "beam_cfg", "beam_moe_workspace_size", "beam_moe_route",
+           "beam_moe_forward", "beam_moe_forward_routed", "beam_moe_forward_traced",
+           "beam_moe_check"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbeam_moe.so")
+
+OP_ROUTE = 0
+OP_FORWARD = 1
+N_STAGES = 7
+STAGE_NAMES = ("router_gemm", "router_topk", "scan", "permute", "gateup_gemm", "down_gemm",
+               "combine")
+
+
+class BeamMoeCfg(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32),
+                ("n_experts", ctypes.c_int32), ("n_group", ctypes.c_int32),
+                ("topk_group", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("renormalize", ctypes.c_int32), ("bias_mode", ctypes.c_int32),
+                ("routed_scale", ctypes.c_float)]
+
+
+class BeamMoeError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {lib().beam_moe_status_string(status).decode()} ({status})")
+
+
+_lib = None
+_P = ctypes.c_void_p
+_CFG = ctypes.POINTER(BeamMoeCfg)
+_SIGS = {
+    "beam_moe_workspace_size": [_CFG, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)],
+    "beam_moe_route": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "beam_moe_forward": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                         ctypes.c_size_t, _P],
+    "beam_moe_forward_routed": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P,
+                                ctypes.c_size_t, _P],
+    "beam_moe_forward_traced": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                ctypes.c_size_t, _P, _P],
+    "beam_moe_trace_create": [ctypes.c_int32, ctypes.POINTER(_P)],
+    "beam_moe_trace_destroy": [_P],
+    "beam_moe_trace_reset": [_P],
+    "beam_moe_trace_read": [_P, _P, ctypes.POINTER(ctypes.c_int32)],
+    "beam_moe_check": [_P, ctypes.c_size_t, _P, ctypes.POINTER(ctypes.c_uint32)],
+    "beam_moe_status_string": [ctypes.c_int],
+}
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libbeam_moe.so not built at {LIB_PATH}; run "
+                              "`python -m sparse_moe_layer_beam_b200._build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, args in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_char_p if name == "beam_moe_status_string" else ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def beam_cfg(H=5120, I=2560, E=256, G=8, Gk=4, K=8, renormalize=True, bias_mode=0, scale=2.5):
+    """Configuration struct; the defaults are the Beam block."""
+    return BeamMoeCfg(H, I, E, G, Gk, K, 1 if renormalize else 0, bias_mode, scale)
+
+
+def _check(status, where):
+    if status != 0:
+        raise BeamMoeError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def beam_moe_workspace_size(cfg, T, op=OP_FORWARD):
+    n = ctypes.c_size_t(0)
+    _check(lib().beam_moe_workspace_size(ctypes.byref(cfg), T, op, ctypes.byref(n)),
+           "beam_moe_workspace_size")
+    return n.value
+
+
+def beam_moe_route(cfg, x, w_router, bias, topk_ids, topk_w, expert_counts, ws, stream=None):
+    T = x.shape[0] if x is not None else 0
+    _check(lib().beam_moe_route(ctypes.byref(cfg), T, _ptr(x), _ptr(w_router), _ptr(bias),
+                                _ptr(topk_ids), _ptr(topk_w), _ptr(expert_counts), _ptr(ws),
+                                ws.numel() * ws.element_size(), _stream(stream)), "beam_moe_route")
+
+
+def beam_moe_forward(cfg, x, w_router, bias, w13, w2, out, ws, topk_ids=None, topk_w=None,
+                     expert_counts=None, stream=None):
+    T = x.shape[0]
+    _check(lib().beam_moe_forward(ctypes.byref(cfg), T, _ptr(x), _ptr(w_router), _ptr(bias),
+                                  _ptr(w13), _ptr(w2), _ptr(out), _ptr(topk_ids), _ptr(topk_w),
+                                  _ptr(expert_counts), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream(stream)), "beam_moe_forward")
+
+
+def beam_moe_forward_traced(cfg, x, w_router, bias, w13, w2, out, ws, trace, topk_ids=None,
+                            topk_w=None, expert_counts=None, stream=None):
+    T = x.shape[0]
+    _check(lib().beam_moe_forward_traced(ctypes.byref(cfg), T, _ptr(x), _ptr(w_router),
+                                         _ptr(bias), _ptr(w13), _ptr(w2), _ptr(out),
+                                         _ptr(topk_ids), _ptr(topk_w), _ptr(expert_counts),
+                                         _ptr(ws), ws.numel() * ws.element_size(),
+                                         _stream(stream), trace.handle),
+           "beam_moe_forward_traced")
+
+
+def beam_moe_forward_routed(cfg, x, topk_ids, topk_w, w13, w2, out, ws, expert_counts=None,
+                            stream=None):
+    T = x.shape[0]
+    _check(lib().beam_moe_forward_routed(ctypes.byref(cfg), T, _ptr(x), _ptr(topk_ids),
+                                         _ptr(topk_w), _ptr(w13), _ptr(w2), _ptr(out),
+                                         _ptr(expert_counts), _ptr(ws),
+                                         ws.numel() * ws.element_size(), _stream(stream)),
+           "beam_moe_forward_routed")
+
+
+def beam_moe_check(ws, stream=None):
+    """Synchronizes the stream, returns the device status bits (0 = clean) and
+    clears them. Raises BeamMoeError on a CUDA error."""
+    flags = ctypes.c_uint32(0)
+    st = lib().beam_moe_check(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream),
+                              ctypes.byref(flags))
+    if st not in (0, 6):
+        raise BeamMoeError(st, "beam_moe_check")
+    return flags.value
+
+
+class Trace:
+    """Per-stage CUDA-event timing of traced forward calls."""
+
+    def __init__(self, capacity):
+        h = _P()
+        _check(lib().beam_moe_trace_create(capacity, ctypes.byref(h)), "beam_moe_trace_create")
+        self.handle = h
+        self.capacity = capacity
+
+    def reset(self):
+        _check(lib().beam_moe_trace_reset(self.handle), "beam_moe_trace_reset")
+
+    def read(self):
+        """List (one entry per traced call) of per-stage milliseconds."""
+        n = ctypes.c_int32(0)
+        buf = (ctypes.c_float * (self.capacity * N_STAGES))()
+        _check(lib().beam_moe_trace_read(self.handle, buf, ctypes.byref(n)), "beam_moe_trace_read")
+        return [list(buf[i * N_STAGES:(i + 1) * N_STAGES]) for i in range(n.value)]
+
+    def close(self):
+        if self.handle:
+            lib().beam_moe_trace_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,422 @@
+// api.cu - host side of the C ABI declared in include/beam_moe.h: argument
+// validation, the workspace layout, TMA descriptor encoding and the launch
+// sequence of one Beam MoE block forward. Nothing here allocates device
+// memory; nothing here synchronizes except beam_moe_check / trace reads.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <initializer_list>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "internal.h"
+
+extern "C" BEAM_MOE_API beam_moe_status beam_moe_workspace_size(const beam_moe_cfg*, int64_t, beam_moe_op,
+                                                   size_t*);
+
+namespace beam {
+
+int device_sm_count() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0)
+      sms = 148;
+    cached[dev] = sms;
+  }
+  return cached[dev];
+}
+
+int router_split_k(int64_t T, int H, int E, int sms);
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Token tile of the grouped GEMMs: the smallest supported N that covers about
+// 1.25x the mean rows per expert (T K / E), so most experts need one tile.
+static int pick_bn(int64_t T, int K, int E) {
+  const double mean = (double)T * K / E;
+  const int opts[5] = {16, 32, 64, 128, 256};
+  for (int b : opts)
+    if (b >= 1.25 * mean) return b;
+  return 256;
+}
+
+Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms) {
+  Layout L;
+  memset(&L, 0, sizeof(L));
+  const int E = c.n_experts, K = c.top_k, H = c.hidden, I = c.inter;
+  L.T = T;
+  L.A = T * K;
+  L.nchunks = (int)((T + kChunk - 1) / kChunk);
+  L.split_k = router_split_k(T, H, E, sms);
+  L.bn = pick_bn(T, K, E);
+  size_t o = 0;
+  auto take = [&](size_t bytes, size_t align) {
+    o = align_up(o, align);
+    size_t at = o;
+    o += bytes;
+    return at;
+  };
+  L.status = take(256, 256);
+  L.counts = take(sizeof(int32_t) * E, 256);
+  L.offsets = take(sizeof(int32_t) * (E + 1), 256);
+  L.nb_off = take(sizeof(int32_t) * (E + 1), 256);
+  L.ids = take(sizeof(int32_t) * (size_t)L.A, 256);
+  L.w = take(sizeof(float) * (size_t)L.A, 256);
+  L.pos = take(sizeof(int32_t) * (size_t)L.A, 256);
+  L.chunk_cnt = take(sizeof(int32_t) * (size_t)L.nchunks * E, 256);
+  L.chunk_mask = take(sizeof(uint32_t) * (size_t)L.nchunks * E * kChunkWords, 256);
+  L.logits = take(sizeof(float) * (size_t)L.split_k * T * E, 256);
+  L.route_end = align_up(o, 256);
+  L.xp = take(2 * (size_t)L.A * H, 1024);
+  L.h = take(2 * (size_t)L.A * I, 1024);
+  L.total = align_up(o, 256);
+  return L;
+}
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][cols], box {box_cols, box_rows}, 128-byte swizzle,
+// zero fill outside the tensor.
+cudaError_t encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                                uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace beam
+
+using beam::Layout;
+
+// ------------------------------------------------------------- validation
+static beam_moe_status check_cfg(const beam_moe_cfg* c) {
+  if (!c) return BEAM_MOE_ERR_INVALID_ARG;
+  if (c->hidden <= 0 || c->inter <= 0 || c->n_experts <= 0 || c->n_group <= 0 ||
+      c->topk_group <= 0 || c->top_k <= 0)
+    return BEAM_MOE_ERR_INVALID_ARG;
+  if (c->renormalize != 0 && c->renormalize != 1) return BEAM_MOE_ERR_INVALID_ARG;
+  if (c->bias_mode != 0 && c->bias_mode != 1) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!isfinite(c->routed_scale)) return BEAM_MOE_ERR_INVALID_ARG;
+  if (c->n_experts % c->n_group != 0 || c->topk_group > c->n_group) return BEAM_MOE_ERR_INVALID_ARG;
+  const int gs = c->n_experts / c->n_group;
+  if (c->top_k > c->topk_group * gs) return BEAM_MOE_ERR_INVALID_ARG;
+  if (c->hidden % 128 != 0 || c->inter % 128 != 0) return BEAM_MOE_ERR_UNSUPPORTED_SHAPE;
+  if (c->hidden > 65536 || c->inter > 65536) return BEAM_MOE_ERR_UNSUPPORTED_SHAPE;
+  if (c->n_experts > 512 || c->top_k > 32 || gs < 2) return BEAM_MOE_ERR_UNSUPPORTED_SHAPE;
+  // the top-k warp gives each lane `per` consecutive experts of one group
+  const int E = c->n_experts;
+  const int per = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : E <= 256 ? 8 : 16;
+  if (gs % per != 0) return BEAM_MOE_ERR_UNSUPPORTED_SHAPE;
+  const int lg = gs / per;
+  if (lg > 32 || (lg & (lg - 1)) != 0) return BEAM_MOE_ERR_UNSUPPORTED_SHAPE;
+  return BEAM_MOE_OK;
+}
+
+static beam_moe_status check_T(const beam_moe_cfg* c, int64_t T) {
+  if (T < 0) return BEAM_MOE_ERR_INVALID_ARG;
+  // permuted rows are addressed with 32-bit ints and TMA row coordinates
+  if (T * (int64_t)c->top_k > (int64_t)1 << 30) return BEAM_MOE_ERR_UNSUPPORTED_SHAPE;
+  return BEAM_MOE_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define BEAM_TRY(expr)                          \
+  do {                                          \
+    beam_moe_status s_ = (expr);                \
+    if (s_ != BEAM_MOE_OK) return s_;           \
+  } while (0)
+
+#define BEAM_CUDA(expr)                         \
+  do {                                          \
+    if ((expr) != cudaSuccess) return BEAM_MOE_ERR_CUDA; \
+  } while (0)
+
+// ------------------------------------------------------------------ trace
+struct beam_moe_trace {
+  int capacity;
+  int n;
+  std::vector<cudaEvent_t> ev;  // capacity * (stages + 1)
+};
+
+namespace {
+
+struct Recorder {
+  beam_moe_trace* tr;
+  cudaStream_t st;
+  int slot;
+  bool on;
+  Recorder(beam_moe_trace* t, cudaStream_t s) : tr(t), st(s), slot(-1), on(false) {
+    if (tr && tr->n < tr->capacity) {
+      slot = tr->n;
+      on = true;
+    }
+  }
+  cudaError_t mark(int i) {
+    if (!on) return cudaSuccess;
+    return cudaEventRecord(tr->ev[(size_t)slot * (BEAM_MOE_N_STAGES + 1) + i], st);
+  }
+  void done() {
+    if (on) tr->n++;
+  }
+};
+
+// Host-only checks, run before any CUDA call: configuration, T, workspace
+// pointer, alignment and size. The size bound is the device-independent one
+// beam_moe_workspace_size reports.
+beam_moe_status common_checks(const beam_moe_cfg* cfg, int64_t T, void* ws, size_t ws_bytes,
+                              beam_moe_op op) {
+  BEAM_TRY(check_cfg(cfg));
+  BEAM_TRY(check_T(cfg, T));
+  if (T == 0) return BEAM_MOE_OK;
+  if (!ws) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return BEAM_MOE_ERR_ALIGNMENT;
+  size_t need = 0;
+  BEAM_TRY(beam_moe_workspace_size(cfg, T, op, &need));
+  if (ws_bytes < need) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status check_ptrs(std::initializer_list<const void*> required,
+                           std::initializer_list<const void*> optional) {
+  for (const void* p : required)
+    if (!p) return BEAM_MOE_ERR_INVALID_ARG;
+  for (const void* p : required)
+    if (!aligned16(p)) return BEAM_MOE_ERR_ALIGNMENT;
+  for (const void* p : optional)
+    if (p && !aligned16(p)) return BEAM_MOE_ERR_ALIGNMENT;
+  return BEAM_MOE_OK;
+}
+
+// Layout for the current device (the first CUDA call of every entry point).
+beam_moe_status plan(const beam_moe_cfg* cfg, int64_t T, Layout* L) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
+  *L = beam::make_layout(*cfg, T, beam::device_sm_count());
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status expert_path(const beam_moe_cfg* cfg, const Layout& L, const uint16_t* x,
+                            const uint16_t* w13, const uint16_t* w2, uint16_t* out,
+                            int32_t* counts_out, char* ws, cudaStream_t st, Recorder& rec) {
+  BEAM_CUDA(beam::launch_scan(*cfg, L, ws, counts_out, st));
+  BEAM_CUDA(rec.mark(3));
+  BEAM_CUDA(beam::launch_permute(*cfg, L, x, ws, st));
+  BEAM_CUDA(rec.mark(4));
+  BEAM_CUDA(beam::launch_gateup(*cfg, L, w13, ws, st));
+  BEAM_CUDA(rec.mark(5));
+  BEAM_CUDA(beam::launch_down(*cfg, L, w2, ws, st));
+  BEAM_CUDA(rec.mark(6));
+  BEAM_CUDA(beam::launch_combine(*cfg, L, out, ws, st));
+  BEAM_CUDA(rec.mark(7));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status forward_impl(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                             const float* w_router, const float* bias, const uint16_t* w13,
+                             const uint16_t* w2, uint16_t* out, int32_t* topk_ids, float* topk_w,
+                             int32_t* expert_counts, void* ws, size_t ws_bytes, void* stream,
+                             beam_moe_trace* trace) {
+  BEAM_TRY(common_checks(cfg, T, ws, ws_bytes, BEAM_MOE_OP_FORWARD));
+  if (T == 0) return BEAM_MOE_OK;
+  BEAM_TRY(check_ptrs({x, w_router, w13, w2, out}, {bias, topk_ids, topk_w, expert_counts}));
+  Layout L;
+  BEAM_TRY(plan(cfg, T, &L));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  Recorder rec(trace, st);
+  BEAM_CUDA(cudaMemsetAsync(w + L.status, 0, 256, st));
+  BEAM_CUDA(rec.mark(0));
+  BEAM_CUDA(beam::launch_router_logits(*cfg, L, x, w_router, w, st));
+  BEAM_CUDA(rec.mark(1));
+  BEAM_CUDA(beam::launch_router_topk(*cfg, L, bias, w, st));
+  BEAM_CUDA(rec.mark(2));
+  BEAM_TRY(expert_path(cfg, L, x, w13, w2, out, expert_counts, w, st, rec));
+  BEAM_CUDA(beam::launch_copy_routes(*cfg, L, topk_ids, topk_w, w, st));
+  rec.done();
+  return BEAM_MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+beam_moe_status beam_moe_workspace_size(const beam_moe_cfg* cfg, int64_t T, beam_moe_op op,
+                                        size_t* bytes) {
+  BEAM_TRY(check_cfg(cfg));
+  BEAM_TRY(check_T(cfg, T));
+  if (!bytes || (op != BEAM_MOE_OP_ROUTE && op != BEAM_MOE_OP_FORWARD))
+    return BEAM_MOE_ERR_INVALID_ARG;
+  if (T == 0) {
+    *bytes = 0;
+    return BEAM_MOE_OK;
+  }
+  // Sized for the largest split-K any device could pick (148 SMs bound it for
+  // B200; the 1024-SM bound keeps the size valid on any part).
+  Layout L = beam::make_layout(*cfg, T, 1024);
+  *bytes = op == BEAM_MOE_OP_ROUTE ? L.route_end : L.total;
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_route(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                               const float* w_router, const float* bias, int32_t* topk_ids,
+                               float* topk_w, int32_t* expert_counts, void* ws, size_t ws_bytes,
+                               void* stream) {
+  BEAM_TRY(common_checks(cfg, T, ws, ws_bytes, BEAM_MOE_OP_ROUTE));
+  if (T == 0) return BEAM_MOE_OK;
+  BEAM_TRY(check_ptrs({x, w_router, topk_ids, topk_w}, {bias, expert_counts}));
+  Layout L;
+  BEAM_TRY(plan(cfg, T, &L));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  BEAM_CUDA(cudaMemsetAsync(w + L.status, 0, 256, st));
+  BEAM_CUDA(beam::launch_router_logits(*cfg, L, x, w_router, w, st));
+  BEAM_CUDA(beam::launch_router_topk(*cfg, L, bias, w, st));
+  if (expert_counts) BEAM_CUDA(beam::launch_scan(*cfg, L, w, expert_counts, st));
+  BEAM_CUDA(beam::launch_copy_routes(*cfg, L, topk_ids, topk_w, w, st));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_forward(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                                 const float* w_router, const float* bias, const uint16_t* w13,
+                                 const uint16_t* w2, uint16_t* out, int32_t* topk_ids,
+                                 float* topk_w, int32_t* expert_counts, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  return forward_impl(cfg, T, x, w_router, bias, w13, w2, out, topk_ids, topk_w, expert_counts,
+                      ws, ws_bytes, stream, nullptr);
+}
+
+beam_moe_status beam_moe_forward_traced(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                                        const float* w_router, const float* bias,
+                                        const uint16_t* w13, const uint16_t* w2, uint16_t* out,
+                                        int32_t* topk_ids, float* topk_w,
+                                        int32_t* expert_counts, void* ws, size_t ws_bytes,
+                                        void* stream, beam_moe_trace* trace) {
+  if (!trace) return BEAM_MOE_ERR_INVALID_ARG;
+  return forward_impl(cfg, T, x, w_router, bias, w13, w2, out, topk_ids, topk_w, expert_counts,
+                      ws, ws_bytes, stream, trace);
+}
+
+beam_moe_status beam_moe_forward_routed(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                                        const int32_t* topk_ids, const float* topk_w,
+                                        const uint16_t* w13, const uint16_t* w2, uint16_t* out,
+                                        int32_t* expert_counts, void* ws, size_t ws_bytes,
+                                        void* stream) {
+  BEAM_TRY(common_checks(cfg, T, ws, ws_bytes, BEAM_MOE_OP_FORWARD));
+  if (T == 0) return BEAM_MOE_OK;
+  BEAM_TRY(check_ptrs({x, topk_ids, topk_w, w13, w2, out}, {expert_counts}));
+  Layout L;
+  BEAM_TRY(plan(cfg, T, &L));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  BEAM_CUDA(cudaMemsetAsync(w + L.status, 0, 256, st));
+  BEAM_CUDA(beam::launch_routes_given(*cfg, L, topk_ids, topk_w, w, st));
+  Recorder none(nullptr, st);
+  return expert_path(cfg, L, x, w13, w2, out, expert_counts, w, st, none);
+}
+
+beam_moe_status beam_moe_trace_create(int32_t capacity, beam_moe_trace** out) {
+  if (!out || capacity <= 0 || capacity > (1 << 20)) return BEAM_MOE_ERR_INVALID_ARG;
+  beam_moe_trace* t = new (std::nothrow) beam_moe_trace;
+  if (!t) return BEAM_MOE_ERR_INVALID_ARG;
+  t->capacity = capacity;
+  t->n = 0;
+  t->ev.assign((size_t)capacity * (BEAM_MOE_N_STAGES + 1), nullptr);
+  for (auto& e : t->ev) {
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      e = nullptr;
+      beam_moe_trace_destroy(t);
+      return BEAM_MOE_ERR_CUDA;
+    }
+  }
+  *out = t;
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_trace_destroy(beam_moe_trace* t) {
+  if (!t) return BEAM_MOE_ERR_INVALID_ARG;
+  for (auto& e : t->ev)
+    if (e) cudaEventDestroy(e);
+  delete t;
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_trace_reset(beam_moe_trace* t) {
+  if (!t) return BEAM_MOE_ERR_INVALID_ARG;
+  t->n = 0;
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_trace_read(beam_moe_trace* t, float* ms, int32_t* n_calls) {
+  if (!t || !n_calls) return BEAM_MOE_ERR_INVALID_ARG;
+  *n_calls = t->n;
+  if (!ms) return BEAM_MOE_OK;
+  for (int i = 0; i < t->n; ++i) {
+    cudaEvent_t* ev = &t->ev[(size_t)i * (BEAM_MOE_N_STAGES + 1)];
+    if (cudaEventSynchronize(ev[BEAM_MOE_N_STAGES]) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
+    for (int s = 0; s < BEAM_MOE_N_STAGES; ++s)
+      if (cudaEventElapsedTime(&ms[(size_t)i * BEAM_MOE_N_STAGES + s], ev[s], ev[s + 1]) !=
+          cudaSuccess)
+        return BEAM_MOE_ERR_CUDA;
+  }
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_check(void* ws, size_t ws_bytes, void* stream, uint32_t* device_flags) {
+  if (!ws || ws_bytes < 256) return BEAM_MOE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
+  uint32_t flags = 0;
+  // The status word is the first 4 bytes of every workspace layout.
+  if (cudaMemcpy(&flags, ws, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return BEAM_MOE_ERR_CUDA;
+  if (cudaMemset(ws, 0, sizeof(flags)) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
+  if (device_flags) *device_flags = flags;
+  return flags ? BEAM_MOE_ERR_DEVICE_TIMEOUT : BEAM_MOE_OK;
+}
+
+const char* beam_moe_status_string(beam_moe_status s) {
+  switch (s) {
+    case BEAM_MOE_OK: return "ok";
+    case BEAM_MOE_ERR_INVALID_ARG: return "invalid argument";
+    case BEAM_MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case BEAM_MOE_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case BEAM_MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case BEAM_MOE_ERR_CUDA: return "CUDA error";
+    case BEAM_MOE_ERR_DEVICE_TIMEOUT: return "device-side check failed (bounded wait or bad id)";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

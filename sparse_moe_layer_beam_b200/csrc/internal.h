@@ -1,0 +1,79 @@
+// internal.h - shared declarations of the Beam MoE block library (not public).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "beam_moe.h"
+
+namespace beam {
+
+// Tokens per dispatch chunk: the stable per-expert rank of a token is counted
+// inside its chunk with one bit per token.
+constexpr int kChunk = 128;
+constexpr int kChunkWords = kChunk / 32;
+
+// Rows of weights per tensor-core tile (the MMA M dimension) and the K step
+// of one pipeline stage (64 bf16 = one 128-byte swizzle row).
+constexpr int kTileM = 128;
+constexpr int kTileK = 64;
+
+// Status bits written by kernels into the workspace status word.
+constexpr uint32_t kFlagProducer = 0x1;
+constexpr uint32_t kFlagMma = 0x2;
+constexpr uint32_t kFlagEpilogue = 0x4;
+constexpr uint32_t kFlagBadExpert = 0x100;
+
+// Byte offsets of every scratch array inside the caller's workspace.
+struct Layout {
+  int64_t T, A;     // tokens, assignments (T * K)
+  int nchunks;      // ceil(T / kChunk)
+  int split_k;      // router split-K factor
+  int bn;           // token tile of the grouped GEMMs
+  size_t status;    // uint32[64]
+  size_t counts;    // int32[E]
+  size_t offsets;   // int32[E + 1] first row of each expert in the permuted rows
+  size_t nb_off;    // int32[E + 1] prefix of ceil(count / bn)
+  size_t ids;       // int32[T * K]
+  size_t w;         // float[T * K]
+  size_t pos;       // int32[T * K] permuted row of each assignment
+  size_t chunk_cnt; // int32[nchunks * E] per-chunk counts, then per-chunk bases
+  size_t chunk_mask;// uint32[nchunks * E * kChunkWords]
+  size_t logits;    // float[split_k * T * E] partial router logits
+  size_t route_end; // bytes needed by the routing op
+  size_t xp;        // bf16[A * H] permuted rows; reused for the down output y
+  size_t h;         // bf16[A * I] SwiGLU activations
+  size_t total;     // bytes needed by the forward op
+};
+
+Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms);
+
+// ---- launchers (each enqueues on `st`, returns cudaGetLastError()) --------
+cudaError_t launch_router_logits(const beam_moe_cfg& c, const Layout& L, const uint16_t* x,
+                                 const float* w_router, char* ws, cudaStream_t st);
+cudaError_t launch_router_topk(const beam_moe_cfg& c, const Layout& L, const float* bias,
+                               char* ws, cudaStream_t st);
+cudaError_t launch_routes_given(const beam_moe_cfg& c, const Layout& L, const int32_t* ids,
+                                const float* w, char* ws, cudaStream_t st);
+cudaError_t launch_scan(const beam_moe_cfg& c, const Layout& L, char* ws, int32_t* counts_out,
+                        cudaStream_t st);
+cudaError_t launch_permute(const beam_moe_cfg& c, const Layout& L, const uint16_t* x, char* ws,
+                           cudaStream_t st);
+cudaError_t launch_gateup(const beam_moe_cfg& c, const Layout& L, const uint16_t* w13, char* ws,
+                          cudaStream_t st);
+cudaError_t launch_down(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2, char* ws,
+                        cudaStream_t st);
+cudaError_t launch_combine(const beam_moe_cfg& c, const Layout& L, uint16_t* out, char* ws,
+                           cudaStream_t st);
+cudaError_t launch_copy_routes(const beam_moe_cfg& c, const Layout& L, int32_t* ids_out,
+                               float* w_out, char* ws, cudaStream_t st);
+
+// Tensor-map encoding through the driver entry point (no link to libcuda).
+cudaError_t encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                                uint32_t box_cols, uint32_t box_rows);
+
+int device_sm_count();
+
+}  // namespace beam

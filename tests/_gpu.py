@@ -1,0 +1,99 @@
+"""GPU-side helpers for parity tests and the smoke check: device buffers filled
+by the synthetic generator, a forward call through the C ABI, and the oracle
+comparison on sampled tokens. Expected values come only from oracle/."""
+import numpy as np
+import torch
+
+import oracle
+import sparse_moe_layer_beam_b200 as bm
+import synth
+from tests import _inputs
+
+TOL = 2e-2  # max |err| <= TOL * RMS(oracle output): bf16 weights/activations, fp32 accumulation
+
+_weights = {}
+
+
+def cfg_of(wl, renormalize=None, bias_mode=0):
+    return bm.beam_cfg(wl.H, wl.I, wl.E, wl.G, wl.Gk, wl.K,
+                       wl.renormalize if renormalize is None else renormalize, bias_mode, wl.scale)
+
+
+def stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def device_weights(wl):
+    """(w13, w2, w_router) on the device, filled on the GPU with the host
+    generator's bytes; cached per block shape (all Beam workloads share them)."""
+    key = (wl.H, wl.I, wl.E)
+    if key not in _weights:
+        _weights.clear()
+        torch.cuda.empty_cache()
+        w13 = torch.empty(wl.w13_elems, dtype=torch.int16, device="cuda")
+        w2 = torch.empty(wl.w2_elems, dtype=torch.int16, device="cuda")
+        synth.dev_w13(wl, w13.data_ptr(), stream())
+        synth.dev_w2(wl, w2.data_ptr(), stream())
+        wr = torch.from_numpy(synth.host_router(wl)).cuda()
+        torch.cuda.synchronize()
+        _weights[key] = (w13, w2, wr)
+    return _weights[key]
+
+
+def to_dev_bits(a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def bits_of(t):
+    return t.cpu().numpy().view(np.uint16)
+
+
+def forward(wl, x_bits, bias=None, renormalize=None, bias_mode=0, weights=None):
+    """Runs beam_moe_forward; returns dict of host arrays and the device flags."""
+    cfg = cfg_of(wl, renormalize, bias_mode)
+    w13, w2, wr = weights if weights is not None else device_weights(wl)
+    T = x_bits.shape[0]
+    x = to_dev_bits(x_bits)
+    b = None if bias is None else torch.from_numpy(np.asarray(bias, np.float32)).cuda()
+    out = torch.empty((T, wl.H), dtype=torch.int16, device="cuda")
+    ids = torch.empty((T, wl.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, wl.K), dtype=torch.float32, device="cuda")
+    counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+    ws = torch.empty(max(bm.beam_moe_workspace_size(cfg, T), 256), dtype=torch.uint8,
+                     device="cuda")
+    bm.beam_moe_forward(cfg, x, wr, b, w13, w2, out, ws, ids, w, counts)
+    flags = bm.beam_moe_check(ws)
+    return {"out": bits_of(out), "ids": ids.cpu().numpy(), "w": w.cpu().numpy(),
+            "counts": counts.cpu().numpy(), "flags": flags}
+
+
+def sorted_routes(ids, w):
+    order = np.argsort(ids, axis=1, kind="stable")
+    return np.take_along_axis(ids, order, 1), np.take_along_axis(w, order, 1)
+
+
+def check_routes(r_gpu, r_oracle, E):
+    """Bit-exact expert sets per token and counts; weights to 1e-6 relative."""
+    gi, gw = sorted_routes(r_gpu["ids"], r_gpu["w"])
+    oi, ow = sorted_routes(r_oracle["ids"], r_oracle["weights"])
+    assert np.array_equal(gi, oi), np.nonzero(np.any(gi != oi, axis=1))[0][:10]
+    assert np.array_equal(r_gpu["counts"], np.bincount(oi.ravel(), minlength=E))
+    assert np.allclose(gw, ow, rtol=1e-6, atol=1e-7)
+
+
+def oracle_outputs(wl, x_bits, tokens, r_oracle, batch=4):
+    """Oracle output rows for the listed tokens, generating only their experts."""
+    cfg = oracle.cfg_for(wl)
+    rows = []
+    for i in range(0, len(tokens), batch):
+        tt = np.asarray(tokens[i:i + batch])
+        ids = r_oracle["ids"][tt]
+        w13, w2 = _inputs.expert_tables(wl, ids)
+        rows.append(oracle.experts(cfg, x_bits[tt], ids, r_oracle["weights"][tt], w13, w2))
+    return np.concatenate(rows, axis=0)
+
+
+def max_rel_err(out_bits, ref):
+    got = synth.bf16_to_f32(out_bits).astype(np.float64)
+    rms = np.sqrt(np.mean(ref ** 2))
+    return np.abs(got - ref).max() / rms, rms

@@ -1,0 +1,182 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Routing must match bit-exactly: the same expert set for every token and the
+same per-expert counts (inputs are re-drawn until every oracle top-k margin
+exceeds 1e-4, so fp32 and fp64 routing must agree). Outputs must match within
+max |err| <= 2e-2 x RMS of the oracle output (bf16 weights and activations,
+fp32 accumulation, bf16 h / y / out). Full-size workloads are compared on all
+routes and on sampled output rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_moe_layer_beam_b200 as bm
+import synth
+from tests import _gpu, _inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_case(name, n_sample):
+    wl = synth.workload(name)
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    g = _gpu.forward(wl, x, bias=b)
+    assert g["flags"] == 0
+    _gpu.check_routes(g, r, wl.E)
+    tokens = synth.sample_tokens(wl.T, n_sample)
+    ref = _gpu.oracle_outputs(wl, x, tokens, r)
+    err, rms = _gpu.max_rel_err(g["out"][tokens], ref)
+    assert err <= _gpu.TOL, (name, err, rms)
+    return wl, x, r, g
+
+
+def test_device_generator_matches_host():
+    wl = synth.workload("decode")
+    n = 1 << 20
+    d = torch.empty(n, dtype=torch.int16, device="cuda")
+    synth.dev_normal_bf16(d.data_ptr(), n, synth.STREAM_W13, _gpu.stream(), idx0=7 * n,
+                          sigma=wl.sigma_w)
+    host = synth.host_normal_bf16(n, synth.STREAM_W13, idx0=7 * n, sigma=wl.sigma_w)
+    assert np.array_equal(_gpu.bits_of(d), host)
+    f = torch.empty(n, dtype=torch.float32, device="cuda")
+    synth.dev_normal_f32(f.data_ptr(), n, synth.STREAM_WROUTER, _gpu.stream(), sigma=wl.sigma_r)
+    assert np.array_equal(f.cpu().numpy(), synth.host_normal_f32(n, synth.STREAM_WROUTER,
+                                                                   sigma=wl.sigma_r))
+    lg = synth.workload("long").with_T(40)
+    xd = torch.empty((40, lg.H), dtype=torch.int16, device="cuda")
+    att = torch.arange(40, dtype=torch.int32, device="cuda") % 3
+    synth.dev_x(lg, xd.data_ptr(), _gpu.stream(), att.data_ptr())
+    assert np.array_equal(_gpu.bits_of(xd), synth.host_x(lg, att.cpu().numpy()))
+
+
+def test_tiny_forward_matches_oracle_everywhere():
+    wl = synth.workload("tiny")
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    g = _gpu.forward(wl, x)
+    assert g["flags"] == 0
+    _gpu.check_routes(g, r, wl.E)
+    cfg = oracle.cfg_for(wl)
+    ref = oracle.experts(cfg, x, r["ids"], r["weights"], synth.host_w13(wl), synth.host_w2(wl))
+    err, _ = _gpu.max_rel_err(g["out"], ref)
+    assert err <= _gpu.TOL, err
+
+
+@pytest.mark.parametrize("T", [1, 7, 129, 300])
+def test_tiny_ragged_token_counts(T):
+    """Ragged T: partial chunks (128 tokens), partial router tiles (64), single token."""
+    wl = synth.workload("tiny").with_T(T)
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    g = _gpu.forward(wl, x)
+    assert g["flags"] == 0
+    _gpu.check_routes(g, r, wl.E)
+    ref = oracle.experts(oracle.cfg_for(wl), x, r["ids"], r["weights"], synth.host_w13(wl),
+                         synth.host_w2(wl))
+    err, _ = _gpu.max_rel_err(g["out"], ref)
+    assert err <= _gpu.TOL, err
+
+
+def test_tie_case_is_bit_exact():
+    """Zero router weights: every score is exactly 0.5; groups 0..Gk-1 and
+    experts 0..K-1 are chosen, each with weight S/K."""
+    for name in ("tiny", "decode"):
+        wl = synth.workload(name).with_T(70)
+        w13, w2, _ = _gpu.device_weights(wl)
+        wr0 = torch.zeros((wl.E, wl.H), dtype=torch.float32, device="cuda")
+        g = _gpu.forward(wl, synth.host_x(wl), weights=(w13, w2, wr0))
+        assert np.array_equal(g["ids"], np.tile(np.arange(wl.K), (wl.T, 1)))
+        assert np.all(g["w"] == np.float32(wl.scale / wl.K))
+        assert np.array_equal(g["counts"][:wl.K], np.full(wl.K, wl.T))
+
+
+def test_renormalize_off_and_selection_only_bias():
+    wl = synth.workload("tiny")
+    x, _, wr, _, r = _inputs.routed_inputs(wl)
+    g = _gpu.forward(wl, x, renormalize=False)
+    r0 = oracle.route(oracle.cfg_for(wl, renormalize=False), x, wr)
+    _gpu.check_routes(g, r0, wl.E)
+    bias = np.zeros(wl.E, np.float32)
+    bias[[1, 2, 9]] = [0.3, 0.2, -0.25]
+    for mode in (0, 1):
+        ocfg = oracle.cfg_for(wl, bias_mode=mode)
+        rb = oracle.route(ocfg, x, wr, bias)
+        ok = rb["margins"].min(1) >= _inputs.MARGIN  # compare tokens with a clear margin
+        g = _gpu.forward(wl, x, bias=bias, bias_mode=mode)
+        sub = {k: v[ok] for k, v in g.items() if k in ("ids", "w")}
+        gi, gw = _gpu.sorted_routes(sub["ids"], sub["w"])
+        oi, ow = _gpu.sorted_routes(rb["ids"][ok], rb["weights"][ok])
+        assert ok.mean() > 0.8
+        assert np.array_equal(gi, oi)
+        assert np.allclose(gw, ow, rtol=1e-6, atol=1e-7)
+
+
+def test_forward_is_deterministic():
+    wl = synth.workload("tiny").with_T(200)
+    x = synth.host_x(wl)
+    a = _gpu.forward(wl, x)
+    b = _gpu.forward(wl, x)
+    assert np.array_equal(a["out"], b["out"]) and np.array_equal(a["w"], b["w"])
+
+
+def test_routed_forward_matches_oracle():
+    """Caller-supplied routes (routing replay): the oracle's own ids and weights."""
+    wl = synth.workload("tiny").with_T(150)
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    cfg = _gpu.cfg_of(wl)
+    w13, w2, _ = _gpu.device_weights(wl)
+    xd = _gpu.to_dev_bits(x)
+    ids = torch.from_numpy(r["ids"]).cuda()
+    w = torch.from_numpy(r["weights"].astype(np.float32)).cuda()
+    out = torch.empty((wl.T, wl.H), dtype=torch.int16, device="cuda")
+    counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+    ws = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T), dtype=torch.uint8, device="cuda")
+    bm.beam_moe_forward_routed(cfg, xd, ids, w, w13, w2, out, ws, counts)
+    assert bm.beam_moe_check(ws) == 0
+    ref = oracle.experts(oracle.cfg_for(wl), x, r["ids"], r["weights"], synth.host_w13(wl),
+                         synth.host_w2(wl))
+    err, _ = _gpu.max_rel_err(_gpu.bits_of(out), ref)
+    assert err <= _gpu.TOL
+    assert np.array_equal(counts.cpu().numpy(), np.bincount(r["ids"].ravel(), minlength=wl.E))
+    # an out-of-range id is dropped and flagged, never dereferenced
+    ids[3, 1] = wl.E + 5
+    bm.beam_moe_forward_routed(cfg, xd, ids, w, w13, w2, out, ws, counts)
+    assert bm.beam_moe_check(ws) & 0x100
+
+
+def test_route_only_entry_point():
+    wl = synth.workload("decode").with_T(300)
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    cfg = _gpu.cfg_of(wl)
+    _, _, wrd = _gpu.device_weights(wl)
+    ids = torch.empty((wl.T, wl.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.K), dtype=torch.float32, device="cuda")
+    counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+    ws = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T, bm.OP_ROUTE), dtype=torch.uint8,
+                     device="cuda")
+    bm.beam_moe_route(cfg, _gpu.to_dev_bits(x), wrd, None, ids, w, counts, ws)
+    assert bm.beam_moe_check(ws) == 0
+    g = {"ids": ids.cpu().numpy(), "w": w.cpu().numpy(), "counts": counts.cpu().numpy()}
+    _gpu.check_routes(g, r, wl.E)
+    # listed by descending score: the oracle's order where consecutive scores differ clearly
+    s = np.take_along_axis(r["scores"], np.argsort(-r["scores"], 1), 1)
+    clear = np.all(np.abs(np.diff(s, axis=1)) > 1e-5, axis=1)
+    assert np.array_equal(g["ids"][clear], r["ids"][clear])
+
+
+def test_decode_full_size():
+    _full_case("decode", 16)
+
+
+def test_prefill_full_size():
+    _full_case("prefill", 24)
+
+
+def test_skewed_full_size():
+    wl, x, r, g = _full_case("skewed", 24)
+    hot = synth.hot_experts(wl)
+    assert g["counts"][hot].sum() > 0.5 * wl.T * wl.K  # the 16 hot experts take most rows
+
+
+def test_long_full_size():
+    _full_case("long", 24)
