@@ -44,6 +44,31 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 STAGES = ("router_gemm", "router_topk", "scan", "permute", "gateup_gemm", "down_gemm", "combine")
 KERNELS_PER_STEP = 7
+GEMM_SOURCES = ("sparse_moe_layer_beam_b200/csrc/grouped_gemm.cu",
+                "sparse_moe_layer_beam_b200/csrc/sm100.cuh")
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the gate/up
+# kernel per touched expert, from the ncu capture summarised in
+# profiles/grouped_gemm_decode_E32_T8.md; valid only for the decode workload and
+# only while the kernel sources hash to `sources_sha256`.
+GATEUP_TRAFFIC = {"workload": "decode", "bytes_per_touched_expert": 52577769,
+                  "sources_sha256": "9c01b80f91c9c3639d6c3ca64250045da96228fbe551422d2c82f01468ae11bc"}
+
+
+def gemm_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gateup_traffic(wl, touched):
+    rec = GATEUP_TRAFFIC
+    if (rec["bytes_per_touched_expert"] is None or wl.name != rec["workload"]
+            or gemm_sources_sha256() != rec["sources_sha256"]):
+        return None
+    return rec["bytes_per_touched_expert"] * touched
 
 
 def describe(wl):
@@ -203,6 +228,22 @@ def run_reference(args, wl):
 
 # -------------------------------------------------------------------------- ours
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (the one collective of a run)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def rank_seed(rank):
+    """Seed of a rank's token batch; all ranks share the expert weights (seed 0)."""
+    return synth.SEED + rank
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
@@ -233,7 +274,7 @@ def run_ours(args, wl):
     bias = synth.host_bias(wl)
     b = None if bias is None else torch.from_numpy(bias).to(dev)
     x = torch.empty((wl.T, wl.H), dtype=torch.int16, device=dev)
-    synth.dev_x(wl, x.data_ptr(), st, seed=synth.SEED + rank)
+    synth.dev_x(wl, x.data_ptr(), st, seed=rank_seed(rank))
     out = torch.empty((wl.T, wl.H), dtype=torch.int16, device=dev)
     counts = torch.zeros(wl.E, dtype=torch.int32, device=dev)
     ws = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T), dtype=torch.uint8, device=dev)
@@ -296,10 +337,7 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(c) for a, c in e2e_ev)
 
-    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
     ms_step = total_ms / args.steps
     tokens = wl.T * world
@@ -322,7 +360,8 @@ def run_ours(args, wl):
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = gateup_traffic(wl, alg["touched_experts"])
+    roof["algorithmic_bytes"] = alg["gateup_bytes"]
     roof["kernel"] = "gateup_grouped_gemm"
     roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
         else "fallback"
@@ -367,10 +406,19 @@ def main():
     ap.add_argument("--workload", default="decode", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (small profiling captures only)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override the expert count, 8 groups kept (small profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
     wl = synth.workload(args.workload)
+    if args.tokens is not None:
+        wl = wl.with_T(args.tokens)
+    if args.experts is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, name=f"{wl.name} (E={args.experts})", E=args.experts)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

@@ -73,7 +73,8 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms) {
   L.chunk_mask = take(sizeof(uint32_t) * (size_t)L.nchunks * E * kChunkWords, 256);
   L.logits = take(sizeof(float) * (size_t)L.split_k * T * E, 256);
   L.route_end = align_up(o, 256);
-  L.xp = take(2 * (size_t)L.A * H, 1024);
+  // permuted rows (bf16) during gate/up, then the down output y (fp32)
+  L.xp = take(4 * (size_t)L.A * H, 1024);
   L.h = take(2 * (size_t)L.A * I, 1024);
   L.total = align_up(o, 256);
   return L;

@@ -13,8 +13,8 @@
 //            earlier tokens of the chunk routed to e (a popcount of the chunk
 //            bits): rows of an expert are in ascending token order. Copies
 //            x[t] to each of its K rows with 16-byte loads and stores.
-//   combine  out[t] = sum_k w[t][k] * y[row(t, k)], k ascending, FP32
-//            accumulation, rounded once to bf16. No atomics.
+//   combine  out[t] = sum_k w[t][k] * y[row(t, k)], k ascending, FP32 y and
+//            FP32 accumulation, rounded once to bf16. No atomics.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -110,21 +110,12 @@ __global__ void __launch_bounds__(128) permute_kernel(const uint16_t* __restrict
   }
 }
 
-__device__ __forceinline__ void unpack8(const uint4& d, float (&f)[8]) {
-  const uint32_t w[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   const __nv_bfloat16 a = __float2bfloat16_rn(lo), b = __float2bfloat16_rn(hi);
   return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
 }
 
-__global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict__ y, int H, int K,
+__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ y, int H, int K,
                                                       const int32_t* __restrict__ pos,
                                                       const float* __restrict__ w,
                                                       uint16_t* __restrict__ out) {
@@ -144,8 +135,9 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict
     for (int k = 0; k < K; ++k) {
       const int p = s_pos[k];
       if (p < 0) continue;
-      float f[8];
-      unpack8(__ldg(reinterpret_cast<const uint4*>(y + (size_t)p * H) + v), f);
+      const float4* src = reinterpret_cast<const float4*>(y + (size_t)p * H) + 2 * v;
+      const float4 a = __ldg(src), b = __ldg(src + 1);
+      const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
       const float wk = s_w[k];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk, f[i], acc[i]);
@@ -179,7 +171,7 @@ cudaError_t launch_permute(const beam_moe_cfg& c, const Layout& L, const uint16_
 cudaError_t launch_combine(const beam_moe_cfg& c, const Layout& L, uint16_t* out, char* ws,
                            cudaStream_t st) {
   combine_kernel<<<(unsigned)L.T, 128, 0, st>>>(
-      reinterpret_cast<const uint16_t*>(ws + L.xp), c.hidden, c.top_k,
+      reinterpret_cast<const float*>(ws + L.xp), c.hidden, c.top_k,
       reinterpret_cast<const int32_t*>(ws + L.pos), reinterpret_cast<const float*>(ws + L.w), out);
   return cudaGetLastError();
 }

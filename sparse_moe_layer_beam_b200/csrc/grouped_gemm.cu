@@ -5,7 +5,7 @@
 //
 //   gate/up:  [g | u] = W13_e x   for every row routed to expert e,
 //             h = silu(g) * u in FP32, stored bf16          (K = H)
-//   down:     y = W2_e h                                      (K = I)
+//   down:     y = W2_e h, stored fp32                         (K = I)
 //
 // Design (sm_100a):
 //  - Swap-AB: 128 weight rows are the MMA M dimension and the routed tokens of
@@ -36,7 +36,7 @@ struct GemmParams {
   const int32_t* counts;  // [E] rows routed to each expert
   const int32_t* offsets; // [E + 1] first permuted row of each expert
   const int32_t* nb_off;  // [E + 1] prefix of token blocks per expert
-  uint16_t* out;          // [A][out_ld] bf16 output rows
+  void* out;              // [A][out_ld] output rows: bf16 h (gate/up), fp32 y (down)
   int64_t out_ld;
   int E;
   int nk;       // K / 64
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
       const int64_t row0 = __ldg(p.offsets + e) + nb * BN;
-      uint16_t* outp = p.out + row0 * p.out_ld + mb * kTileM + r;
+      const int64_t o0 = row0 * p.out_ld + mb * kTileM + r;
       for (int c0 = 0; c0 < n_mma; c0 += 16) {
         uint32_t g[16], u[16];
         tmem_ld16(tb + c0, g);
@@ -256,9 +256,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 16; ++j) {
           const int t = c0 + j;
           if (t < rows) {
-            const float v = GATEUP ? silu_mul(__uint_as_float(g[j]), __uint_as_float(u[j]))
-                                   : __uint_as_float(g[j]);
-            outp[(int64_t)t * p.out_ld] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            if (GATEUP) {
+              const float v = silu_mul(__uint_as_float(g[j]), __uint_as_float(u[j]));
+              static_cast<uint16_t*>(p.out)[o0 + (int64_t)t * p.out_ld] =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            } else {
+              static_cast<float*>(p.out)[o0 + (int64_t)t * p.out_ld] = __uint_as_float(g[j]);
+            }
           }
         }
       }
@@ -332,7 +336,7 @@ cudaError_t launch_gateup(const beam_moe_cfg& c, const Layout& L, const uint16_t
   err = encode_tmap_2d_bf16(&tx, ws + L.xp, (uint64_t)H, (uint64_t)L.A, kTileK, (uint32_t)L.bn);
   if (err != cudaSuccess) return err;
   GemmParams p = base_params(c, L, ws);
-  p.out = reinterpret_cast<uint16_t*>(ws + L.h);
+  p.out = ws + L.h;
   p.out_ld = I;
   p.nk = H / kTileK;
   p.w_rows = 2 * I;
@@ -350,7 +354,7 @@ cudaError_t launch_down(const beam_moe_cfg& c, const Layout& L, const uint16_t* 
   err = encode_tmap_2d_bf16(&tx, ws + L.h, (uint64_t)I, (uint64_t)L.A, kTileK, (uint32_t)L.bn);
   if (err != cudaSuccess) return err;
   GemmParams p = base_params(c, L, ws);
-  p.out = reinterpret_cast<uint16_t*>(ws + L.xp);  // y reuses the permuted-input rows
+  p.out = ws + L.xp;  // fp32 y reuses the permuted-input rows
   p.out_ld = H;
   p.nk = I / kTileK;
   p.w_rows = H;

@@ -43,7 +43,7 @@ struct Layout {
   size_t chunk_mask;// uint32[nchunks * E * kChunkWords]
   size_t logits;    // float[split_k * T * E] partial router logits
   size_t route_end; // bytes needed by the routing op
-  size_t xp;        // bf16[A * H] permuted rows; reused for the down output y
+  size_t xp;        // bf16[A * H] permuted rows; reused for the down output y, fp32[A * H]
   size_t h;         // bf16[A * I] SwiGLU activations
   size_t total;     // bytes needed by the forward op
 };

@@ -73,12 +73,15 @@ def sorted_routes(ids, w):
 
 
 def check_routes(r_gpu, r_oracle, E):
-    """Bit-exact expert sets per token and counts; weights to 1e-6 relative."""
+    """Bit-exact expert sets per token and counts; weights to 1e-5 relative: the
+    fp32 router logit is a sequential sum over H = 5120 products, whose rounding
+    error reaches a few 1e-6, times the sigmoid slope (<= 1/4), relative to
+    weights of about 0.3."""
     gi, gw = sorted_routes(r_gpu["ids"], r_gpu["w"])
     oi, ow = sorted_routes(r_oracle["ids"], r_oracle["weights"])
     assert np.array_equal(gi, oi), np.nonzero(np.any(gi != oi, axis=1))[0][:10]
     assert np.array_equal(r_gpu["counts"], np.bincount(oi.ravel(), minlength=E))
-    assert np.allclose(gw, ow, rtol=1e-6, atol=1e-7)
+    assert np.allclose(gw, ow, rtol=1e-5, atol=1e-6)
 
 
 def oracle_outputs(wl, x_bits, tokens, r_oracle, batch=4):

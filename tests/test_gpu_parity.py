@@ -4,7 +4,7 @@ Routing must match bit-exactly: the same expert set for every token and the
 same per-expert counts (inputs are re-drawn until every oracle top-k margin
 exceeds 1e-4, so fp32 and fp64 routing must agree). Outputs must match within
 max |err| <= 2e-2 x RMS of the oracle output (bf16 weights and activations,
-fp32 accumulation, bf16 h / y / out). Full-size workloads are compared on all
+fp32 accumulation, bf16 h, fp32 y, bf16 out). Full-size workloads are compared on all
 routes and on sampled output rows.
 """
 import numpy as np
@@ -108,7 +108,7 @@ def test_renormalize_off_and_selection_only_bias():
         oi, ow = _gpu.sorted_routes(rb["ids"][ok], rb["weights"][ok])
         assert ok.mean() > 0.8
         assert np.array_equal(gi, oi)
-        assert np.allclose(gw, ow, rtol=1e-6, atol=1e-7)
+        assert np.allclose(gw, ow, rtol=1e-5, atol=1e-6)
 
 
 def test_forward_is_deterministic():
