@@ -102,6 +102,37 @@ BEAM_MOE_API beam_moe_status beam_moe_route(const beam_moe_cfg* cfg, int64_t T, 
                                void* stream);
 
 /*
+ * Routing without any device allocation and without a caller workspace. The
+ * paper has no counterpart: this entry point exists for callers that cannot
+ * call cudaMalloc, for example a serving process whose memory pool has already
+ * reserved the GPU's memory for weights and caches, or a runtime that forbids
+ * device allocations once it has started. The caller still passes inputs and
+ * outputs exactly as for beam_moe_route (same meaning, layout and alignment);
+ * the scratch is a fixed BEAM_MOE_NOALLOC_SCRATCH_BYTES array inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.
+ *  - Limits: T <= BEAM_MOE_NOALLOC_MAX_TOKENS and n_experts <=
+ *    BEAM_MOE_NOALLOC_MAX_EXPERTS; larger calls return
+ *    BEAM_MOE_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *  - The first call on a device looks up the array's device address for that
+ *    device (once, with that device current); make that first call before
+ *    any stream capture on the device.
+ *  - Every call on a device shares the one array: calls that may overlap on
+ *    the GPU (different streams, no ordering between them) race and must be
+ *    serialized by the caller.
+ *  - Results equal beam_moe_route's up to the order of FP32 partial sums of
+ *    the router logits (the number of H splits may differ).
+ */
+#define BEAM_MOE_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+#define BEAM_MOE_NOALLOC_MAX_TOKENS 2048
+#define BEAM_MOE_NOALLOC_MAX_EXPERTS 256
+BEAM_MOE_API beam_moe_status beam_moe_route_noalloc(const beam_moe_cfg* cfg, int64_t T,
+                                                    const uint16_t* x, const float* w_router,
+                                                    const float* bias, int32_t* topk_ids,
+                                                    float* topk_w, int32_t* expert_counts,
+                                                    void* stream);
+
+/*
  * Whole block forward: routing as beam_moe_route, then for every token
  *   out[t] = sum_k topk_w[t][k] * Wd_e (silu(Wg_e x_t) * (Wu_e x_t)),  e = topk_ids[t][k]
  * ("Welcome Beam", section "Mixture of Experts": SwiGLU experts of

@@ -16,6 +16,7 @@ import os
 
 __all__ = ["BeamMoeCfg", "BeamMoeError", "Trace", "OP_ROUTE", "OP_FORWARD", "N_STAGES",
            "STAGE_NAMES", "lib", "beam_cfg", "beam_moe_workspace_size", "beam_moe_route",
+           "beam_moe_route_noalloc",
            "beam_moe_forward", "beam_moe_forward_routed", "beam_moe_forward_traced",
            "beam_moe_check"]
 
@@ -49,6 +50,7 @@ _CFG = ctypes.POINTER(BeamMoeCfg)
 _SIGS = {
     "beam_moe_workspace_size": [_CFG, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)],
     "beam_moe_route": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "beam_moe_route_noalloc": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P],
     "beam_moe_forward": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                          ctypes.c_size_t, _P],
     "beam_moe_forward_routed": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -113,6 +115,18 @@ def beam_moe_route(cfg, x, w_router, bias, topk_ids, topk_w, expert_counts, ws, 
     _check(lib().beam_moe_route(ctypes.byref(cfg), T, _ptr(x), _ptr(w_router), _ptr(bias),
                                 _ptr(topk_ids), _ptr(topk_w), _ptr(expert_counts), _ptr(ws),
                                 ws.numel() * ws.element_size(), _stream(stream)), "beam_moe_route")
+
+
+def beam_moe_route_noalloc(cfg, x, w_router, bias, topk_ids, topk_w, expert_counts=None,
+                           stream=None):
+    """Routing with the library's fixed scratch instead of a workspace, for
+    callers that cannot allocate device memory (at most 2048 tokens and 256
+    experts; concurrent calls on one device race)."""
+    T = x.shape[0]
+    _check(lib().beam_moe_route_noalloc(ctypes.byref(cfg), T, _ptr(x), _ptr(w_router),
+                                        _ptr(bias), _ptr(topk_ids), _ptr(topk_w),
+                                        _ptr(expert_counts), _stream(stream)),
+           "beam_moe_route_noalloc")
 
 
 def beam_moe_forward(cfg, x, w_router, bias, w13, w2, out, ws, topk_ids=None, topk_w=None,
