@@ -55,6 +55,9 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms) {
   L.nchunks = (int)((T + kChunk - 1) / kChunk);
   L.split_k = router_split_k(T, H, E, sms);
   L.bn = pick_bn(T, K, E);
+  // CTA pairs once experts average at least one full 256-token block: below
+  // that the GEMMs stream weights and one CTA per tile is enough.
+  L.pair = (L.bn == 256 && (double)T * K / E >= 256.0 && pair_gemm_supported(c)) ? 1 : 0;
   size_t o = 0;
   auto take = [&](size_t bytes, size_t align) {
     o = align_up(o, align);
@@ -111,6 +114,24 @@ cudaError_t encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t col
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// W13 [E][2I][H] seen as 5-D {H, 16, 2, I/16, E} (k, row in a 16-row block,
+// gate/up, block, expert): a box {64, 16, 2, 4, 1} lands in shared memory as
+// 128 rows ordered gate 0-15, up 0-15, gate 16-31, up 16-31, ... of 64
+// consecutive intermediate indices.
+cudaError_t encode_tmap_w13_interleaved(CUtensorMap* map, const void* w13, uint64_t H, uint64_t I,
+                                        uint64_t E) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[5] = {H, 16, 2, I / 16, E};
+  const cuuint64_t strides[4] = {H * 2, I * H * 2, 16 * H * 2, 2 * I * H * 2};
+  const cuuint32_t box[5] = {64, 16, 2, 4, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(w13), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -235,9 +256,11 @@ beam_moe_status expert_path(const beam_moe_cfg* cfg, const Layout& L, const uint
   BEAM_CUDA(rec.mark(3));
   BEAM_CUDA(beam::launch_permute(*cfg, L, x, ws, st));
   BEAM_CUDA(rec.mark(4));
-  BEAM_CUDA(beam::launch_gateup(*cfg, L, w13, ws, st));
+  BEAM_CUDA(L.pair ? beam::launch_gateup_pair(*cfg, L, w13, ws, st)
+                   : beam::launch_gateup(*cfg, L, w13, ws, st));
   BEAM_CUDA(rec.mark(5));
-  BEAM_CUDA(beam::launch_down(*cfg, L, w2, ws, st));
+  BEAM_CUDA(L.pair ? beam::launch_down_pair(*cfg, L, w2, ws, st)
+                   : beam::launch_down(*cfg, L, w2, ws, st));
   BEAM_CUDA(rec.mark(6));
   BEAM_CUDA(beam::launch_combine(*cfg, L, out, ws, st));
   BEAM_CUDA(rec.mark(7));

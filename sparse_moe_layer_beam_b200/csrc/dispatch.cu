@@ -5,7 +5,8 @@
 // normalized weights and scaled by 2.5); grouping rows by expert so that every
 // expert runs as one dense GEMM is this library's design.
 //
-//   scan     per-expert counts, first row of each expert (exclusive scan),
+//   scan     per-expert counts (popcounts of the chunk bits), first row of
+//            each expert (exclusive scan),
 //            the base row of every (chunk, expert) and the prefix of token
 //            tiles per expert that the grouped GEMMs schedule from. All of it
 //            stays on the device.
@@ -22,14 +23,50 @@
 namespace beam {
 namespace {
 
-__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_cnt, int nchunks,
+__device__ __forceinline__ int chunk_count(const uint32_t* __restrict__ bits, size_t i) {
+  const uint4 m = __ldg(reinterpret_cast<const uint4*>(bits) + i);
+  return __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
+}
+
+// Exclusive scan of v over threads 0..n-1 (n <= 1024); every thread of the
+// block must call it. Returns the exclusive prefix, writes the total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += n;
+  }
+  if (lane == 31) warp_tot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += n;
+    }
+    warp_tot[lane] = wi - w;  // exclusive prefix of each warp
+    if (lane == 31) *total = wi;
+  }
+  __syncthreads();
+  const int r = warp_tot[warp] + inc - v;
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(1024) scan_kernel(const uint32_t* __restrict__ bits,
+                                                    int32_t* __restrict__ chunk_base, int nchunks,
                                                     int E, int bn, int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ nb_off,
                                                     int32_t* __restrict__ counts_out) {
-  __shared__ int32_t part[1024];
-  __shared__ int32_t s_off[513];
-  __shared__ int32_t s_nb[513];
+  __shared__ int32_t part[1024];   // per (team member, expert) partial counts
+  __shared__ int32_t s_off[512];   // first row of each expert
+  __shared__ int32_t warp_tot[32];
+  __shared__ int32_t total[2];
   const int tid = threadIdx.x;
   const int tpe = 1024 / E;  // threads per expert (E <= 512)
   const int e = tid % E, j = tid / E;
@@ -38,21 +75,24 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_
   const int c0 = j * L, c1 = min(nchunks, c0 + L);
   int sum = 0;
   if (act)
-    for (int c = c0; c < c1; ++c) sum += chunk_cnt[(size_t)c * E + e];
+    for (int c = c0; c < c1; ++c) sum += chunk_count(bits, (size_t)c * E + e);
   part[tid] = sum;
   __syncthreads();
+  int tot = 0;
+  if (tid < E)
+    for (int q = 0; q < tpe; ++q) tot += part[q * E + tid];
+  const int off = block_exclusive_scan(tid < E ? tot : 0, warp_tot, &total[0]);
+  const int nbo = block_exclusive_scan(tid < E ? (tot + bn - 1) / bn : 0, warp_tot, &total[1]);
+  if (tid < E) {
+    s_off[tid] = off;
+    offsets[tid] = off;
+    nb_off[tid] = nbo;
+    counts[tid] = tot;
+    if (counts_out) counts_out[tid] = tot;
+  }
   if (tid == 0) {
-    int run = 0, nrun = 0;
-    for (int x = 0; x < E; ++x) {
-      int tot = 0;
-      for (int q = 0; q < tpe; ++q) tot += part[q * E + x];
-      s_off[x] = run;
-      s_nb[x] = nrun;
-      run += tot;
-      nrun += (tot + bn - 1) / bn;
-    }
-    s_off[E] = run;
-    s_nb[E] = nrun;
+    offsets[E] = total[0];
+    nb_off[E] = total[1];
   }
   __syncthreads();
   if (act) {
@@ -60,17 +100,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_
     for (int q = 0; q < j; ++q) run += part[q * E + e];
     for (int c = c0; c < c1; ++c) {
       const size_t i = (size_t)c * E + e;
-      const int v = chunk_cnt[i];
-      chunk_cnt[i] = run;
-      run += v;
-    }
-  }
-  for (int x = tid; x <= E; x += 1024) {
-    offsets[x] = s_off[x];
-    nb_off[x] = s_nb[x];
-    if (x < E) {
-      counts[x] = s_off[x + 1] - s_off[x];
-      if (counts_out) counts_out[x] = s_off[x + 1] - s_off[x];
+      chunk_base[i] = run;
+      run += chunk_count(bits, i);
     }
   }
 }
@@ -151,7 +182,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
 
 cudaError_t launch_scan(const beam_moe_cfg& c, const Layout& L, char* ws, int32_t* counts_out,
                         cudaStream_t st) {
-  scan_kernel<<<1, 1024, 0, st>>>(reinterpret_cast<int32_t*>(ws + L.chunk_cnt), L.nchunks,
+  scan_kernel<<<1, 1024, 0, st>>>(reinterpret_cast<const uint32_t*>(ws + L.chunk_mask),
+                                  reinterpret_cast<int32_t*>(ws + L.chunk_cnt), L.nchunks,
                                   c.n_experts, L.bn, reinterpret_cast<int32_t*>(ws + L.counts),
                                   reinterpret_cast<int32_t*>(ws + L.offsets),
                                   reinterpret_cast<int32_t*>(ws + L.nb_off), counts_out);

@@ -26,33 +26,20 @@
 //    after its own copies and MMAs have completed.
 #include <cuda_bf16.h>
 
+#include "grouped_gemm.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
 namespace beam {
 namespace {
 
-struct GemmParams {
-  const int32_t* counts;  // [E] rows routed to each expert
-  const int32_t* offsets; // [E + 1] first permuted row of each expert
-  const int32_t* nb_off;  // [E + 1] prefix of token blocks per expert
-  void* out;              // [A][out_ld] output rows: bf16 h (gate/up), fp32 y (down)
-  int64_t out_ld;
-  int E;
-  int nk;       // K / 64
-  int w_rows;   // weight rows per expert (2I or H)
-  int up_rows;  // row offset of the up projection inside an expert (I)
-  int n_mblk;   // 128-row weight blocks per expert (I / 128 or H / 128)
-  unsigned* status;
-};
+using gg::GemmParams;
+using gg::decode_tile;
+using gg::pow2_at_least;
+using gg::silu_mul;
+
 
 constexpr int kThreads = 192;
-
-__host__ __device__ constexpr int pow2_at_least(int v) {
-  int p = 32;
-  while (p < v) p <<= 1;
-  return p;
-}
 
 template <bool GATEUP, int BN>
 struct Cfg {
@@ -71,28 +58,6 @@ struct Cfg {
   static_assert(kTmemCols <= 512, "TMEM overflow");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "bad BN");
 };
-
-// Tile -> (expert, weight block, token block). The largest e with
-// nb_off[e] * n_mblk <= tile is never an empty expert.
-__device__ __forceinline__ void decode_tile(int tile, const GemmParams& p, int& e, int& mb,
-                                            int& nb) {
-  int lo = 0, hi = p.E - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(p.nb_off + mid) * p.n_mblk <= tile) lo = mid;
-    else hi = mid - 1;
-  }
-  e = lo;
-  const int base = __ldg(p.nb_off + e);
-  const int nblk = __ldg(p.nb_off + e + 1) - base;
-  const int local = tile - base * p.n_mblk;
-  mb = local / nblk;
-  nb = local - mb * nblk;
-}
-
-__device__ __forceinline__ float silu_mul(float g, float u) {
-  return g / (1.0f + __expf(-g)) * u;
-}
 
 template <bool GATEUP, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -140,8 +105,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------ TMA producer
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();
+      // Weights are streamed once when an expert has a single token block;
+      // otherwise every token block's CTA reads the same weight tile, and it
+      // must stay in L2 until they all have.
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       int64_t issued = 0;
@@ -151,6 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         decode_tile(tile, p, e, mb, nb);
         const int wrow = e * p.w_rows + mb * kTileM;
         const int xrow = __ldg(p.offsets + e) + nb * BN;
+        const int nblk = __ldg(p.nb_off + e + 1) - __ldg(p.nb_off + e);
+        const uint64_t pol_w = nblk == 1 ? pol_stream : pol_keep;
         for (int kb = 0; kb < p.nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, kFlagProducer)) {
             ok = false;
@@ -162,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (GATEUP)
             tma_load_2d(sa + C::kABytes, &tm_w, &full[stage], kb * kTileK, wrow + p.up_rows,
                         pol_w);
-          tma_load_2d(sa + C::kNA * C::kABytes, &tm_x, &full[stage], kb * kTileK, xrow, pol_x);
+          tma_load_2d(sa + C::kNA * C::kABytes, &tm_x, &full[stage], kb * kTileK, xrow, pol_keep);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;

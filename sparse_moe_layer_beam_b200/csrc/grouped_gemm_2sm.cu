@@ -1,0 +1,348 @@
+// grouped_gemm_2sm.cu - the expert GEMMs for many rows per expert, on CTA
+// pairs (tcgen05 cta_group::2). Same operations as grouped_gemm.cu:
+//
+//   gate/up:  [g | u] = W13_e x, h = silu(g) * u in FP32 -> bf16   (K = H)
+//   down:     y = W2_e h -> fp32                                  (K = I)
+//
+// One MMA covers 256 weight rows x up to 256 tokens. Each CTA of the pair
+// holds 128 weight rows and half of the tokens in its shared memory and 128
+// accumulator rows in its TMEM, so a CTA moves a third fewer operand bytes per
+// FLOP than a single-CTA 128 x 256 tile, and the 128 x 256 FP32 accumulator
+// (256 TMEM columns) is double-buffered: the epilogue of one tile overlaps the
+// MMAs of the next.
+//
+// Gate/up rows are interleaved in 16-row blocks inside a CTA's 128 rows
+// (gate 0-15, up 0-15, gate 16-31, ...), loaded with one 5-D TMA box, so that
+// a warp's 32 TMEM lanes hold 16 gate rows and the 16 up rows of the same
+// intermediate indices; lanes exchange halves with one shuffle.
+//
+// Roles (both CTAs have the same warps): warp 0 issues this CTA's TMA loads,
+// whose completion is counted on the even CTA's barrier; warp 1 of the even
+// CTA issues the pair's MMAs and commits to barriers in both CTAs; warps 2-5
+// of each CTA drain their own TMEM and tell the even CTA's MMA thread. The
+// pair allocates TMEM together and meets at a cluster barrier before freeing
+// it. No load uses multicast. Every wait is bounded.
+#include <cuda_bf16.h>
+
+#include "grouped_gemm.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace beam {
+namespace {
+
+using gg::GemmParams;
+using gg::decode_tile;
+using gg::silu_mul;
+
+constexpr int kThreads = 192;
+constexpr int kPairM = 256;  // weight rows per pair tile
+constexpr int kPairN = 256;  // max tokens per pair tile (the token block)
+
+struct PairCfg {
+  static constexpr int kABytes = 128 * kTileK * 2;  // this CTA's 128 weight rows
+  static constexpr int kBBytes = 128 * kTileK * 2;  // this CTA's half of 256 tokens
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = 6;
+  static constexpr int kAccCols = kPairN;  // FP32 accumulator columns per stage
+  static constexpr int kTmemCols = 512;    // two accumulator stages
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+};
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
+                             const __grid_constant__ CUtensorMap tm_x, const GemmParams p) {
+  using C = PairCfg;
+  constexpr int STAGES = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: the CTA that issues MMAs
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);   // the even CTA's arrive.expect_tx + both CTAs' bytes
+      mbar_init(&empty[s], 1);  // one multicast commit per consumed stage
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * 128);  // epilogue threads of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int total = __ldg(p.nb_off + p.E) * p.n_mblk;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_normal();
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += n_pairs) {
+        int e, mb, nb;
+        decode_tile(tile, p, e, mb, nb);
+        const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
+        const int half = ((rows + 15) & ~15) >> 1;
+        const int xrow = __ldg(p.offsets + e) + nb * kPairN + (int)rank * half;
+        const int nblk = __ldg(p.nb_off + e + 1) - __ldg(p.nb_off + e);
+        const uint64_t pol_w = nblk == 1 ? pol_stream : pol_keep;
+        // first weight row of this CTA's 128 (down) or first intermediate
+        // index of its 64 gate/up pairs
+        const int w0 = GATEUP ? mb * 128 + (int)rank * 64
+                              : e * p.w_rows + mb * kPairM + (int)rank * 128;
+        for (int kb = 0; kb < p.nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, kFlagProducer)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::kStageBytes;
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+          const uint32_t bar = mapa_shared(smem_addr(&full[stage]), 0);
+          const int kx = kb * kTileK;
+          if (GATEUP) {
+            tma_load_5d_pair(sa, &tm_w, bar, kx, 0, 0, w0 / 16, e, pol_w);
+          } else {
+            tma_load_2d_pair(sa, &tm_w, bar, kx, w0, pol_w);
+          }
+          tma_load_2d_pair(sa + C::kABytes, &tm_x, bar, kx, xrow, pol_keep);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // The even CTA's full barriers count both CTAs' copies: wait for the
+      // last ones to land before either CTA can leave.
+      if (leader) {
+        const int64_t first = issued > STAGES ? issued - STAGES : 0;
+        for (int64_t i = first; i < issued; ++i)
+          mbar_wait(&full[i % STAGES], (uint32_t)((i / STAGES) & 1), nullptr, nullptr, 0u,
+                    100000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // --------------------------------------------------------- MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += n_pairs) {
+        int e, mb, nb;
+        decode_tile(tile, p, e, mb, nb);
+        const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
+        const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_f32(kPairM, n_mma);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, kFlagMma)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(acc * C::kAccCols);
+        for (int kb = 0; kb < p.nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, kFlagMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
+          const uint64_t da = smem_desc_k_sw128(sa);
+          const uint64_t db = smem_desc_k_sw128(sa + C::kABytes);
+#pragma unroll
+          for (int k4 = 0; k4 < kTileK / 16; ++k4)
+            umma_bf16_pair(d, da + 2u * k4, db + 2u * k4, idesc, (kb | k4) != 0);
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(&tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // Every MMA of the pair completes before TMEM is released.
+      umma_commit_pair(drain, 0x1);
+      mbar_wait(drain, 0, nullptr, nullptr, 0u, 100000000ull);
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quadrant of this warp
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < total; tile += n_pairs) {
+      int e, mb, nb;
+      decode_tile(tile, p, e, mb, nb);
+      const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
+      const int n_mma = (rows + 15) & ~15;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, kFlagEpilogue)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
+      const int64_t row0 = __ldg(p.offsets + e) + nb * kPairN;
+      if (GATEUP) {
+        // lanes 0-15: gate rows, 16-31: up rows of 16 intermediate indices
+        const int idx = mb * 128 + (int)rank * 64 + q * 16 + (lane & 15);
+        const int tsel = (lane >> 4) * 8;  // this lane's half of each 16 tokens
+        uint16_t* out = static_cast<uint16_t*>(p.out) + idx;
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(tb + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t send = lane < 16 ? v[8 + j] : v[j];
+            const float other = __uint_as_float(__shfl_xor_sync(0xffffffffu, send, 16));
+            const float g = lane < 16 ? __uint_as_float(v[j]) : other;
+            const float u = lane < 16 ? other : __uint_as_float(v[8 + j]);
+            const int t = c0 + tsel + j;
+            if (t < rows)
+              out[(row0 + t) * p.out_ld] = __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(g, u)));
+          }
+        }
+      } else {
+        const int col = mb * kPairM + (int)rank * 128 + q * 32 + lane;
+        float* out = static_cast<float*>(p.out) + col;
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(tb + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < rows) out[(row0 + c0 + j) * p.out_ld] = __uint_as_float(v[j]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(mapa_shared(smem_addr(&tempty[acc]), 0));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();  // both CTAs done with TMEM and with each other's memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
+  }
+}
+
+template <bool GATEUP>
+cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p,
+                     cudaStream_t st) {
+  // Per device: the shared-memory attribute and the number of CTA pairs that
+  // can be resident at once (a pair needs two SMs of one GPC). The grid is
+  // exactly that many pairs, so no pair waits for another to finish.
+  static int configured_device = -1;
+  static int resident_pairs = 0;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = PairCfg::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (configured_device != dev) {
+    err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATEUP>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    cfg.gridDim = dim3((unsigned)(device_sm_count() & ~1));
+    int clusters = 0;
+    err = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<GATEUP>, &cfg);
+    if (err != cudaSuccess) return err;
+    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    resident_pairs = clusters < device_sm_count() / 2 ? clusters : device_sm_count() / 2;
+    configured_device = dev;
+  }
+  cfg.gridDim = dim3((unsigned)(2 * resident_pairs));
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATEUP>, tw, tx, p);
+}
+
+GemmParams base_params(const beam_moe_cfg& c, const Layout& L, char* ws) {
+  GemmParams p;
+  p.counts = reinterpret_cast<const int32_t*>(ws + L.counts);
+  p.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
+  p.nb_off = reinterpret_cast<const int32_t*>(ws + L.nb_off);
+  p.E = c.n_experts;
+  p.status = reinterpret_cast<unsigned*>(ws + L.status);
+  return p;
+}
+
+}  // namespace
+
+bool pair_gemm_supported(const beam_moe_cfg& c) {
+  return c.hidden % kPairM == 0 && c.inter % 128 == 0;
+}
+
+cudaError_t launch_gateup_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w13,
+                               char* ws, cudaStream_t st) {
+  const int H = c.hidden, I = c.inter, E = c.n_experts;
+  CUtensorMap tw, tx;
+  cudaError_t err = encode_tmap_w13_interleaved(&tw, w13, (uint64_t)H, (uint64_t)I, (uint64_t)E);
+  if (err != cudaSuccess) return err;
+  err = encode_tmap_2d_bf16(&tx, ws + L.xp, (uint64_t)H, (uint64_t)L.A, kTileK, 128);
+  if (err != cudaSuccess) return err;
+  GemmParams p = base_params(c, L, ws);
+  p.out = ws + L.h;
+  p.out_ld = I;
+  p.nk = H / kTileK;
+  p.w_rows = 2 * I;
+  p.up_rows = I;
+  p.n_mblk = I / 128;  // 128 intermediate indices (gate + up) per pair tile
+  return run_pair<true>(tw, tx, p, st);
+}
+
+cudaError_t launch_down_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2,
+                             char* ws, cudaStream_t st) {
+  const int H = c.hidden, I = c.inter, E = c.n_experts;
+  CUtensorMap tw, tx;
+  cudaError_t err = encode_tmap_2d_bf16(&tw, w2, (uint64_t)I, (uint64_t)E * H, kTileK, 128);
+  if (err != cudaSuccess) return err;
+  err = encode_tmap_2d_bf16(&tx, ws + L.h, (uint64_t)I, (uint64_t)L.A, kTileK, 128);
+  if (err != cudaSuccess) return err;
+  GemmParams p = base_params(c, L, ws);
+  p.out = ws + L.xp;  // fp32 y reuses the permuted-input rows
+  p.out_ld = H;
+  p.nk = I / kTileK;
+  p.w_rows = H;
+  p.up_rows = 0;
+  p.n_mblk = H / kPairM;
+  return run_pair<false>(tw, tx, p, st);
+}
+
+}  // namespace beam

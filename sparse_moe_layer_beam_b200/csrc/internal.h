@@ -32,6 +32,7 @@ struct Layout {
   int nchunks;      // ceil(T / kChunk)
   int split_k;      // router split-K factor
   int bn;           // token tile of the grouped GEMMs
+  int pair;         // 1: grouped GEMMs on CTA pairs (many rows per expert)
   size_t status;    // uint32[64]
   size_t counts;    // int32[E]
   size_t offsets;   // int32[E + 1] first row of each expert in the permuted rows
@@ -39,7 +40,7 @@ struct Layout {
   size_t ids;       // int32[T * K]
   size_t w;         // float[T * K]
   size_t pos;       // int32[T * K] permuted row of each assignment
-  size_t chunk_cnt; // int32[nchunks * E] per-chunk counts, then per-chunk bases
+  size_t chunk_cnt; // int32[nchunks * E] first row of each (chunk, expert)
   size_t chunk_mask;// uint32[nchunks * E * kChunkWords]
   size_t logits;    // float[split_k * T * E] partial router logits
   size_t route_end; // bytes needed by the routing op
@@ -65,6 +66,11 @@ cudaError_t launch_gateup(const beam_moe_cfg& c, const Layout& L, const uint16_t
                           cudaStream_t st);
 cudaError_t launch_down(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2, char* ws,
                         cudaStream_t st);
+bool pair_gemm_supported(const beam_moe_cfg& c);
+cudaError_t launch_gateup_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w13,
+                               char* ws, cudaStream_t st);
+cudaError_t launch_down_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2,
+                             char* ws, cudaStream_t st);
 cudaError_t launch_combine(const beam_moe_cfg& c, const Layout& L, uint16_t* out, char* ws,
                            cudaStream_t st);
 cudaError_t launch_copy_routes(const beam_moe_cfg& c, const Layout& L, int32_t* ids_out,
@@ -73,6 +79,9 @@ cudaError_t launch_copy_routes(const beam_moe_cfg& c, const Layout& L, int32_t* 
 // Tensor-map encoding through the driver entry point (no link to libcuda).
 cudaError_t encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                                 uint32_t box_cols, uint32_t box_rows);
+
+cudaError_t encode_tmap_w13_interleaved(CUtensorMap* map, const void* w13, uint64_t H, uint64_t I,
+                                        uint64_t E);
 
 int device_sm_count();
 

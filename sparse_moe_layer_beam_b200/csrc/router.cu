@@ -3,18 +3,20 @@
 // "Residual Stream": the router is computed in FP32).
 //
 // Stage 0 (router_logits_kernel): logits = x W_r^T on CUDA cores in FP32,
-// with an optional split over H so that small batches still fill the GPU.
-// Partial sums are written per split and added in split order by stage 1, so
-// the result does not depend on scheduling.
+// 128 tokens x 128 experts per CTA, 8 x 8 per thread, with an optional split
+// over H (at most 16 parts) so that small batches still fill the GPU. Partial
+// sums are written per split and added in split order by stage 1, so the
+// result does not depend on scheduling. The same kernel clears the dispatch
+// bits that stage 1 sets.
 //
 // Stage 1 (router_topk_kernel): one warp per token. Lane l holds PER
 // consecutive experts; a group of E/G experts spans E/G/PER lanes. The warp
 // computes the sigmoid scores, each group's sum of its two best choice
 // scores, keeps the Gk best groups, picks the K best experts inside them
-// (order key: value descending, expert id ascending) and the combine weights.
-// The same CTA records, for its chunk of tokens, one bit per (expert, token)
-// and the per-expert counts: the dispatch later derives every token's stable
-// row inside its expert from these bits.
+// (order key: value descending, expert id ascending) and the combine weights,
+// and sets one bit per (expert, token) in its 128-token chunk (an OR, so the
+// result does not depend on the order of the warps). The dispatch derives
+// every token's stable row inside its expert from these bits.
 #include <math.h>
 
 #include "internal.h"
@@ -22,56 +24,64 @@
 namespace beam {
 namespace {
 
-constexpr int kRBM = 64;   // tokens per CTA
+constexpr int kRBM = 128;  // tokens per CTA
 constexpr int kRBE = 128;  // experts per CTA
-constexpr int kRBK = 32;   // K per shared-memory stage
+constexpr int kRBK = 16;   // K per shared-memory stage
+constexpr int kMaxSplit = 16;
 
 __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
                                                             const float* __restrict__ wr,
                                                             float* __restrict__ part, int T, int H,
-                                                            int E, int kc) {
+                                                            int E, int kc,
+                                                            uint32_t* __restrict__ bits,
+                                                            int64_t n_bits_words) {
   __shared__ __align__(16) float xs[2][kRBK][kRBM];
   __shared__ __align__(16) float wsm[2][kRBK][kRBE];
   const int tid = threadIdx.x;
+  {  // clear the dispatch bits set by stage 1
+    const int64_t nthreads = (int64_t)gridDim.x * gridDim.y * gridDim.z * blockDim.x;
+    const int64_t cta = ((int64_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    for (int64_t i = cta * blockDim.x + tid; i < n_bits_words; i += nthreads) bits[i] = 0u;
+  }
   const int m0 = blockIdx.x * kRBM, e0 = blockIdx.y * kRBE;
   const int kbeg = blockIdx.z * kc;
-  const int tx = tid & 15, ty = tid >> 4;  // experts {tx*4+q, 64+tx*4+q}, tokens ty*4+i
-
-  // loader mapping: x rows tid&63, k offset (tid>>6)*8; w rows tid&127, k offset (tid>>7)*4+8r
-  const int lx_t = m0 + (tid & 63), lx_k = (tid >> 6) * 8;
-  const int lw_e = e0 + (tid & 127), lw_k = (tid >> 7) * 4;
-  const bool x_ok = lx_t < T, w_ok = lw_e < E;
-  const uint16_t* xrow = x + (size_t)(x_ok ? lx_t : 0) * H;
-  const float* wrow = wr + (size_t)(w_ok ? lw_e : 0) * H;
+  // compute mapping: tokens {ty*4+i, 64+ty*4+i}, experts {tx*4+j, 64+tx*4+j}
+  const int tx = tid & 15, ty = tid >> 4;
+  // loader mapping: x row tid&127 at k offset (tid>>7)*8; w row tid&127 at (tid>>7)*4 and +8
+  const int lrow = tid & 127, lx_k = (tid >> 7) * 8, lw_k = (tid >> 7) * 4;
+  const bool x_ok = m0 + lrow < T, w_ok = e0 + lrow < E;
+  const uint16_t* xrow = x + (size_t)(x_ok ? m0 + lrow : 0) * H;
+  const float* wrow = wr + (size_t)(w_ok ? e0 + lrow : 0) * H;
 
   uint4 xr;
-  float4 wv[4];
+  float4 wv0, wv1;
   auto load = [&](int k0) {
     xr = x_ok ? __ldg(reinterpret_cast<const uint4*>(xrow + k0 + lx_k)) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-      wv[r] = w_ok ? __ldg(reinterpret_cast<const float4*>(wrow + k0 + lw_k + 8 * r))
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    wv0 = w_ok ? __ldg(reinterpret_cast<const float4*>(wrow + k0 + lw_k))
+               : make_float4(0.f, 0.f, 0.f, 0.f);
+    wv1 = w_ok ? __ldg(reinterpret_cast<const float4*>(wrow + k0 + lw_k + 8))
+               : make_float4(0.f, 0.f, 0.f, 0.f);
   };
   auto store = [&](int buf) {
     const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      xs[buf][lx_k + 2 * j][tid & 63] = __uint_as_float(xw[j] << 16);
-      xs[buf][lx_k + 2 * j + 1][tid & 63] = __uint_as_float(xw[j] & 0xFFFF0000u);
+      xs[buf][lx_k + 2 * j][lrow] = __uint_as_float(xw[j] << 16);
+      xs[buf][lx_k + 2 * j + 1][lrow] = __uint_as_float(xw[j] & 0xFFFF0000u);
     }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      wsm[buf][lw_k + 8 * r + 0][tid & 127] = wv[r].x;
-      wsm[buf][lw_k + 8 * r + 1][tid & 127] = wv[r].y;
-      wsm[buf][lw_k + 8 * r + 2][tid & 127] = wv[r].z;
-      wsm[buf][lw_k + 8 * r + 3][tid & 127] = wv[r].w;
-    }
+    wsm[buf][lw_k + 0][lrow] = wv0.x;
+    wsm[buf][lw_k + 1][lrow] = wv0.y;
+    wsm[buf][lw_k + 2][lrow] = wv0.z;
+    wsm[buf][lw_k + 3][lrow] = wv0.w;
+    wsm[buf][lw_k + 8][lrow] = wv1.x;
+    wsm[buf][lw_k + 9][lrow] = wv1.y;
+    wsm[buf][lw_k + 10][lrow] = wv1.z;
+    wsm[buf][lw_k + 11][lrow] = wv1.w;
   };
 
-  float acc[4][8];
+  float acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
@@ -84,13 +94,14 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
     if (it + 1 < nk) load(kbeg + (it + 1) * kRBK);
 #pragma unroll
     for (int k = 0; k < kRBK; ++k) {
-      const float4 a = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 4]);
+      const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][k][64 + ty * 4]);
       const float4 b0 = *reinterpret_cast<const float4*>(&wsm[buf][k][tx * 4]);
       const float4 b1 = *reinterpret_cast<const float4*>(&wsm[buf][k][64 + tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
@@ -100,8 +111,8 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
 
   float* out = part + (size_t)blockIdx.z * T * E;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = m0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int t = m0 + (i >> 2) * 64 + ty * 4 + (i & 3);
     if (t >= T) continue;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -133,126 +144,138 @@ __device__ __forceinline__ void warp_argmax(float& v, int& idx, float& s) {
 }
 
 struct TopkArgs {
-  const float* part;  // [split_k][T][E] partial logits, or NULL (ids given)
+  const float* part;  // [split_k][T][E] partial logits
   int split_k;
   const float* bias;  // [E] or NULL
   int bias_mode;
   int T, E, G, Gk, K, renorm;
   float scale;
-  int32_t* ids;        // [T][K]
-  float* w;            // [T][K]
-  int32_t* chunk_cnt;  // [nchunks][E]
-  uint32_t* chunk_mask;// [nchunks][E][kChunkWords]
+  int32_t* ids;         // [T][K]
+  float* w;             // [T][K]
+  uint32_t* chunk_mask; // [nchunks][E][kChunkWords]
 };
 
+// Sum of the split partial logits of PER consecutive experts, split order.
 template <int PER>
-__global__ void __launch_bounds__(256) router_topk_kernel(TopkArgs a) {
-  __shared__ uint32_t smask[512 * kChunkWords];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int c = blockIdx.x, t0 = c * kChunk;
-  const int E = a.E, K = a.K;
-  for (int i = tid; i < E * kChunkWords; i += 256) smask[i] = 0u;
-  __syncthreads();
-
-  const int gs = E / a.G;          // experts per group
-  const int lg = gs / PER;         // lanes per group (power of two)
-  const bool active = lane * PER < E;
-  const int gid = active ? (lane * PER) / gs : 0x7fffffff;
-
-  for (int tl = warp; tl < kChunk; tl += 8) {
-    const int t = t0 + tl;
-    if (t >= a.T) break;
-    float s[PER], ch[PER];
+__device__ __forceinline__ void load_logits(const float* __restrict__ p, size_t stride, int n,
+                                            float (&l)[PER]) {
 #pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const int e = lane * PER + j;
-      s[j] = 0.f;
-      ch[j] = -INFINITY;
-      if (e < E) {
-        float l = 0.f;
-        for (int sp = 0; sp < a.split_k; ++sp) l += a.part[((size_t)sp * a.T + t) * E + e];
-        const float b = a.bias ? a.bias[e] : 0.f;
-        if (a.bias_mode == 0) l += b;
-        s[j] = 1.0f / (1.0f + expf(-l));
-        ch[j] = a.bias_mode == 1 ? s[j] + b : s[j];
+  for (int j = 0; j < PER; ++j) l[j] = 0.f;
+  if constexpr (PER % 4 == 0) {
+#pragma unroll 4
+    for (int sp = 0; sp < n; ++sp) {
+      const float4* q = reinterpret_cast<const float4*>(p + sp * stride);
+#pragma unroll
+      for (int v = 0; v < PER / 4; ++v) {
+        const float4 f = __ldg(q + v);
+        l[4 * v] += f.x;
+        l[4 * v + 1] += f.y;
+        l[4 * v + 2] += f.z;
+        l[4 * v + 3] += f.w;
       }
     }
-    // group score: sum of the two best choice scores of the group
-    float b1 = -INFINITY, b2 = -INFINITY;
+  } else {
+    for (int sp = 0; sp < n; ++sp)
 #pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      if (ch[j] > b1) {
-        b2 = b1;
-        b1 = ch[j];
-      } else if (ch[j] > b2) {
-        b2 = ch[j];
-      }
-    }
-    for (int off = 1; off < lg; off <<= 1) {
-      const float o1 = __shfl_xor_sync(0xffffffffu, b1, off);
-      const float o2 = __shfl_xor_sync(0xffffffffu, b2, off);
-      const float n2 = fmaxf(fminf(b1, o1), fmaxf(b2, o2));
-      b1 = fmaxf(b1, o1);
-      b2 = n2;
-    }
-    const float gscore = b1 + b2;
-    // keep the Gk best groups
-    bool kept = false;
-    for (int r = 0; r < a.Gk; ++r) {
-      float v = (active && !kept) ? gscore : -INFINITY;
-      int id = gid;
-      float unused = 0.f;
-      warp_argmax(v, id, unused);
-      if (gid == id) kept = true;
-    }
-    // top-K experts inside the kept groups
-    uint32_t taken = 0u;
-    int my_e = -1;
-    float my_s = 0.f, wsum = 0.f;
-    for (int k = 0; k < K; ++k) {
-      float bv = -INFINITY, bs = 0.f;
-      int be = 0x7fffffff;
-      if (kept) {
-#pragma unroll
-        for (int j = 0; j < PER; ++j) {
-          const int e = lane * PER + j;
-          if (e < E && !((taken >> j) & 1u) && (ch[j] > bv || (ch[j] == bv && e < be))) {
-            bv = ch[j];
-            be = e;
-            bs = s[j];
-          }
-        }
-      }
-      warp_argmax(bv, be, bs);
-      if (lane == be / PER) taken |= 1u << (be - lane * PER);
-      if (lane == k) {
-        my_e = be;
-        my_s = bs;
-      }
-      wsum += bs;
-    }
-    if (lane < K) {
-      const float wk = a.renorm ? my_s / wsum : my_s;
-      a.ids[(size_t)t * K + lane] = my_e;
-      a.w[(size_t)t * K + lane] = a.scale * wk;
-      atomicOr(&smask[my_e * kChunkWords + (tl >> 5)], 1u << (tl & 31));
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < E; e += 256) {
-    int cnt = 0;
-#pragma unroll
-    for (int wd = 0; wd < kChunkWords; ++wd) {
-      const uint32_t m = smask[e * kChunkWords + wd];
-      cnt += __popc(m);
-      a.chunk_mask[((size_t)c * E + e) * kChunkWords + wd] = m;
-    }
-    a.chunk_cnt[(size_t)c * E + e] = cnt;
+      for (int j = 0; j < PER; ++j) l[j] += __ldg(p + sp * stride + j);
   }
 }
 
-// Caller-supplied routes: copy ids / weights into the workspace and record the
-// chunk bits and counts. Out-of-range ids are dropped (id -1) and flagged.
+template <int PER>
+__global__ void __launch_bounds__(256) router_topk_kernel(TopkArgs a) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int t = blockIdx.x * 8 + (tid >> 5);
+  if (t >= a.T) return;  // whole warps leave together
+  const int E = a.E, K = a.K;
+  const int gs = E / a.G;   // experts per group
+  const int lg = gs / PER;  // lanes per group (power of two)
+  const bool active = lane * PER < E;
+  const int gid = active ? (lane * PER) / gs : 0x7fffffff;
+
+  float s[PER], ch[PER];
+  if (active) {
+    float l[PER];
+    load_logits<PER>(a.part + (size_t)t * E + lane * PER, (size_t)a.T * E, a.split_k, l);
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int e = lane * PER + j;
+      const float b = a.bias ? a.bias[e] : 0.f;
+      const float lj = a.bias_mode == 0 ? l[j] + b : l[j];
+      s[j] = 1.0f / (1.0f + expf(-lj));
+      ch[j] = a.bias_mode == 1 ? s[j] + b : s[j];
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      s[j] = 0.f;
+      ch[j] = -INFINITY;
+    }
+  }
+  // group score: sum of the two best choice scores of the group
+  float b1 = -INFINITY, b2 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    if (ch[j] > b1) {
+      b2 = b1;
+      b1 = ch[j];
+    } else if (ch[j] > b2) {
+      b2 = ch[j];
+    }
+  }
+  for (int off = 1; off < lg; off <<= 1) {
+    const float o1 = __shfl_xor_sync(0xffffffffu, b1, off);
+    const float o2 = __shfl_xor_sync(0xffffffffu, b2, off);
+    const float n2 = fmaxf(fminf(b1, o1), fmaxf(b2, o2));
+    b1 = fmaxf(b1, o1);
+    b2 = n2;
+  }
+  const float gscore = b1 + b2;
+  // keep the Gk best groups
+  bool kept = false;
+  for (int r = 0; r < a.Gk; ++r) {
+    float v = (active && !kept) ? gscore : -INFINITY;
+    int id = gid;
+    float unused = 0.f;
+    warp_argmax(v, id, unused);
+    if (gid == id) kept = true;
+  }
+  // top-K experts inside the kept groups
+  uint32_t taken = 0u;
+  int my_e = -1;
+  float my_s = 0.f, wsum = 0.f;
+  for (int k = 0; k < K; ++k) {
+    float bv = -INFINITY, bs = 0.f;
+    int be = 0x7fffffff;
+    if (kept) {
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        const int e = lane * PER + j;
+        if (!((taken >> j) & 1u) && (ch[j] > bv || (ch[j] == bv && e < be))) {
+          bv = ch[j];
+          be = e;
+          bs = s[j];
+        }
+      }
+    }
+    warp_argmax(bv, be, bs);
+    if (lane == be / PER) taken |= 1u << (be - lane * PER);
+    if (lane == k) {
+      my_e = be;
+      my_s = bs;
+    }
+    wsum += bs;
+  }
+  if (lane < K) {
+    const float wk = a.renorm ? my_s / wsum : my_s;
+    a.ids[(size_t)t * K + lane] = my_e;
+    a.w[(size_t)t * K + lane] = a.scale * wk;
+    const int c = t / kChunk, tl = t - c * kChunk;
+    atomicOr(&a.chunk_mask[((size_t)c * E + my_e) * kChunkWords + (tl >> 5)], 1u << (tl & 31));
+  }
+}
+
+// Caller-supplied routes: copy ids / weights into the workspace and write the
+// chunk bits. Out-of-range ids are dropped (id -1) and flagged.
 __global__ void __launch_bounds__(256) routes_given_kernel(const int32_t* __restrict__ ids_in,
                                                            const float* __restrict__ w_in,
                                                            TopkArgs a, unsigned* status) {
@@ -277,16 +300,8 @@ __global__ void __launch_bounds__(256) routes_given_kernel(const int32_t* __rest
     a.w[o] = w_in[o];
   }
   __syncthreads();
-  for (int e = tid; e < E; e += 256) {
-    int cnt = 0;
-#pragma unroll
-    for (int wd = 0; wd < kChunkWords; ++wd) {
-      const uint32_t m = smask[e * kChunkWords + wd];
-      cnt += __popc(m);
-      a.chunk_mask[((size_t)c * E + e) * kChunkWords + wd] = m;
-    }
-    a.chunk_cnt[(size_t)c * E + e] = cnt;
-  }
+  for (int i = tid; i < E * kChunkWords; i += 256)
+    a.chunk_mask[(size_t)c * E * kChunkWords + i] = smask[i];
 }
 
 TopkArgs topk_args(const beam_moe_cfg& c, const Layout& L, char* ws) {
@@ -304,21 +319,30 @@ TopkArgs topk_args(const beam_moe_cfg& c, const Layout& L, char* ws) {
   a.scale = c.routed_scale;
   a.ids = reinterpret_cast<int32_t*>(ws + L.ids);
   a.w = reinterpret_cast<float*>(ws + L.w);
-  a.chunk_cnt = reinterpret_cast<int32_t*>(ws + L.chunk_cnt);
   a.chunk_mask = reinterpret_cast<uint32_t*>(ws + L.chunk_mask);
   return a;
 }
 
 }  // namespace
 
+// Split of H for the router GEMM: the divisor of H/16 (at most 16) that
+// minimises waves x work per CTA, with two CTAs resident per SM; ties go to
+// the smaller split (fewer partial sums for stage 1 to read).
 int router_split_k(int64_t T, int H, int E, int sms) {
   const int64_t tiles = ((T + kRBM - 1) / kRBM) * ((E + kRBE - 1) / kRBE);
+  const int64_t slots = 2 * (int64_t)(sms > 0 ? sms : 1);
   const int max_split = H / kRBK;
-  int want = (int)((2 * (int64_t)sms + tiles - 1) / tiles);
-  if (want < 1) want = 1;
   int best = 1;
-  for (int s = 1; s <= max_split; ++s)
-    if (max_split % s == 0 && s <= want) best = s;
+  double best_cost = 1e30;
+  for (int s = 1; s <= max_split && s <= kMaxSplit; ++s) {
+    if (max_split % s != 0) continue;
+    const int64_t waves = (tiles * s + slots - 1) / slots;
+    const double cost = (double)waves / s;
+    if (cost < best_cost - 1e-12) {
+      best_cost = cost;
+      best = s;
+    }
+  }
   return best;
 }
 
@@ -327,8 +351,9 @@ cudaError_t launch_router_logits(const beam_moe_cfg& c, const Layout& L, const u
   const int H = c.hidden, E = c.n_experts;
   dim3 grid((unsigned)((L.T + kRBM - 1) / kRBM), (unsigned)((E + kRBE - 1) / kRBE),
             (unsigned)L.split_k);
-  router_logits_kernel<<<grid, 256, 0, st>>>(x, w_router, reinterpret_cast<float*>(ws + L.logits),
-                                              (int)L.T, H, E, H / L.split_k);
+  router_logits_kernel<<<grid, 256, 0, st>>>(
+      x, w_router, reinterpret_cast<float*>(ws + L.logits), (int)L.T, H, E, H / L.split_k,
+      reinterpret_cast<uint32_t*>(ws + L.chunk_mask), (int64_t)L.nchunks * E * kChunkWords);
   return cudaGetLastError();
 }
 
@@ -337,7 +362,7 @@ cudaError_t launch_router_topk(const beam_moe_cfg& c, const Layout& L, const flo
   TopkArgs a = topk_args(c, L, ws);
   a.bias = bias;
   const int E = c.n_experts;
-  const dim3 grid((unsigned)L.nchunks);
+  const dim3 grid((unsigned)((L.T + 7) / 8));
   if (E <= 32) router_topk_kernel<1><<<grid, 256, 0, st>>>(a);
   else if (E <= 64) router_topk_kernel<2><<<grid, 256, 0, st>>>(a);
   else if (E <= 128) router_topk_kernel<4><<<grid, 256, 0, st>>>(a);

@@ -77,6 +77,21 @@ def test_tiny_ragged_token_counts(T):
     assert err <= _gpu.TOL, err
 
 
+@pytest.mark.parametrize("T", [1024, 1500])
+def test_tiny_many_rows_per_expert(T):
+    """At least 256 rows per expert on average: the grouped GEMMs run on CTA
+    pairs (cta_group::2) with ragged token blocks."""
+    wl = synth.workload("tiny").with_T(T)
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    g = _gpu.forward(wl, x)
+    assert g["flags"] == 0
+    _gpu.check_routes(g, r, wl.E)
+    ref = oracle.experts(oracle.cfg_for(wl), x, r["ids"], r["weights"], synth.host_w13(wl),
+                         synth.host_w2(wl))
+    err, _ = _gpu.max_rel_err(g["out"], ref)
+    assert err <= _gpu.TOL, err
+
+
 def test_tie_case_is_bit_exact():
     """Zero router weights: every score is exactly 0.5; groups 0..Gk-1 and
     experts 0..K-1 are chosen, each with weight S/K."""
