@@ -55,9 +55,14 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms) {
   L.nchunks = (int)((T + kChunk - 1) / kChunk);
   L.split_k = router_split_k(T, H, E, sms);
   L.bn = pick_bn(T, K, E);
-  // CTA pairs once experts average at least one full 256-token block: below
-  // that the GEMMs stream weights and one CTA per tile is enough.
-  L.pair = (L.bn == 256 && (double)T * K / E >= 256.0 && pair_gemm_supported(c)) ? 1 : 0;
+  // CTA pairs halve the token-row bytes each SM reads per weight byte and
+  // double-buffer the accumulator. That pays once experts average 64 rows or
+  // more (measured: prefill at 128 rows is faster on pairs for both GEMMs);
+  // below that the GEMMs stream weights and one CTA per tile is enough.
+  const double mean_rows = (double)T * K / E;
+  const bool pair_ok = L.bn == 256 && pair_gemm_supported(c);
+  L.pair_gateup = (pair_ok && mean_rows >= 64.0) ? 1 : 0;
+  L.pair_down = (pair_ok && mean_rows >= 64.0) ? 1 : 0;
   size_t o = 0;
   auto take = [&](size_t bytes, size_t align) {
     o = align_up(o, align);
@@ -256,10 +261,10 @@ beam_moe_status expert_path(const beam_moe_cfg* cfg, const Layout& L, const uint
   BEAM_CUDA(rec.mark(3));
   BEAM_CUDA(beam::launch_permute(*cfg, L, x, ws, st));
   BEAM_CUDA(rec.mark(4));
-  BEAM_CUDA(L.pair ? beam::launch_gateup_pair(*cfg, L, w13, ws, st)
+  BEAM_CUDA(L.pair_gateup ? beam::launch_gateup_pair(*cfg, L, w13, ws, st)
                    : beam::launch_gateup(*cfg, L, w13, ws, st));
   BEAM_CUDA(rec.mark(5));
-  BEAM_CUDA(L.pair ? beam::launch_down_pair(*cfg, L, w2, ws, st)
+  BEAM_CUDA(L.pair_down ? beam::launch_down_pair(*cfg, L, w2, ws, st)
                    : beam::launch_down(*cfg, L, w2, ws, st));
   BEAM_CUDA(rec.mark(6));
   BEAM_CUDA(beam::launch_combine(*cfg, L, out, ws, st));

@@ -32,7 +32,8 @@ struct Layout {
   int nchunks;      // ceil(T / kChunk)
   int split_k;      // router split-K factor
   int bn;           // token tile of the grouped GEMMs
-  int pair;         // 1: grouped GEMMs on CTA pairs (many rows per expert)
+  int pair_gateup; // 1: gate/up grouped GEMM on CTA pairs
+  int pair_down;   // 1: down grouped GEMM on CTA pairs
   size_t status;    // uint32[64]
   size_t counts;    // int32[E]
   size_t offsets;   // int32[E + 1] first row of each expert in the permuted rows
