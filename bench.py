@@ -50,8 +50,8 @@ GEMM_SOURCES = ("sparse_moe_layer_beam_b200/csrc/grouped_gemm.cu",
 # kernel per touched expert, from the ncu capture summarised in
 # profiles/grouped_gemm_decode_E32_T8.md; valid only for the decode workload and
 # only while the kernel sources hash to `sources_sha256`.
-GATEUP_TRAFFIC = {"workload": "decode", "bytes_per_touched_expert": 52577769,
-                  "sources_sha256": "9c01b80f91c9c3639d6c3ca64250045da96228fbe551422d2c82f01468ae11bc"}
+GATEUP_TRAFFIC = {"workload": "decode", "bytes_per_touched_expert": 52586103,
+                  "sources_sha256": "17de9080793b81c0f1393c5a0e542a9dc3deab90f1bcd27127c54d109320227d"}
 
 
 def gemm_sources_sha256():
@@ -264,7 +264,8 @@ def run_ours(args, wl):
     stream = torch.cuda.current_stream()
     st = stream.cuda_stream
 
-    cfg = bm.beam_cfg(wl.H, wl.I, wl.E, wl.G, wl.Gk, wl.K, wl.renormalize, 0, wl.scale)
+    cfg = bm.beam_cfg(wl.H, wl.I, wl.E, wl.G, wl.Gk, wl.K, wl.renormalize, args.bias_mode,
+                      wl.scale)
     # all ranks hold the same experts (seed 0); each rank routes its own tokens
     w13 = torch.empty(wl.w13_elems, dtype=torch.int16, device=dev)
     w2 = torch.empty(wl.w2_elems, dtype=torch.int16, device=dev)
@@ -281,8 +282,15 @@ def run_ours(args, wl):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
 
+    ids = torch.empty((wl.T, wl.K), dtype=torch.int32, device=dev)
+    wts = torch.empty((wl.T, wl.K), dtype=torch.float32, device=dev)
+    if args.replay:  # record the routes once; the timed steps replay them
+        bm.beam_moe_forward(cfg, x, wr, b, w13, w2, out, ws, ids, wts, counts, stream=st)
+
     def step(trace=None):
-        if trace is None:
+        if args.replay:
+            bm.beam_moe_forward_routed(cfg, x, ids, wts, w13, w2, out, ws, counts, stream=st)
+        elif trace is None:
             bm.beam_moe_forward(cfg, x, wr, b, w13, w2, out, ws, expert_counts=counts,
                                 stream=st)
         else:
@@ -296,7 +304,7 @@ def run_ours(args, wl):
     if flags:
         raise SystemExit(f"device status flags {flags:#x} after warm-up")
 
-    trace = bm.Trace(args.steps)
+    trace = None if args.replay else bm.Trace(args.steps)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     clocks = ClockSampler(local)
@@ -314,7 +322,8 @@ def run_ours(args, wl):
         dist.barrier()
     clk = clocks.stop()
     total_ms = sum(a.elapsed_time(c) for a, c in ev)
-    stage_ms = np.array(trace.read())  # [steps][stages]
+    stage_ms = (np.full((args.steps, len(STAGES)), np.nan) if trace is None
+                else np.array(trace.read()))  # [steps][stages]
     flags = bm.beam_moe_check(ws, st)
     if flags:
         raise SystemExit(f"device status flags {flags:#x} in the timed region")
@@ -346,20 +355,26 @@ def run_ours(args, wl):
 
     alg = algorithmic(wl, counts.cpu().numpy())
     peaks, peak_kind = load_peaks()
-    gate_ms = float(stage_ms[:, 4].mean())
+    # Tensor peak: the burst figure for short steps, the sustained (power-capped)
+    # figure once a step lasts 10 ms or more and the GPU runs at its power cap.
+    sustained = ms_step >= 10.0 and "bf16_tflops_sustained" in peaks
+    tc_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     stage_mean = {n: float(stage_ms[:, i].mean()) for i, n in enumerate(STAGES)}
     # the gate/up grouped GEMM dominates every configuration; its bound follows
     # from its arithmetic intensity (flop per weight byte = rows per expert)
+    gate_ms = float(stage_ms[:, 4].mean()) if trace is not None else float("nan")
     t_hbm = alg["gateup_bytes"] / (peaks["hbm_gbs"] * 1e9)
-    t_tc = alg["gateup_flops"] / (peaks["bf16_tflops"] * 1e12)
+    t_tc = alg["gateup_flops"] / (tc_peak * 1e12)
     if t_hbm >= t_tc:
         achieved = alg["gateup_bytes"] / (gate_ms / 1000.0) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     else:
         achieved = alg["gateup_flops"] / (gate_ms / 1000.0) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                "peak_kind": "sustained" if sustained else "burst"}
+    if args.replay:  # no per-stage events on this entry point
+        roof.update(achieved=None, frac=None)
+    roof["frac"] = None if roof["achieved"] is None else roof["achieved"] / roof["peak"]
     roof["traffic"] = gateup_traffic(wl, alg["touched_experts"])
     roof["algorithmic_bytes"] = alg["gateup_bytes"]
     roof["kernel"] = "gateup_grouped_gemm"
@@ -370,19 +385,24 @@ def run_ours(args, wl):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": describe(wl), "T": wl.T, "tokens_per_rank": wl.T,
+        "config": {"workload": describe(wl) + (" [routes replayed]" if args.replay else "")
+                   + (" [selection-only bias]" if args.bias_mode == 1 else ""),
+                   "T": wl.T, "tokens_per_rank": wl.T,
                    "l2": "flushed before every timed step (256 MB write, outside the events)",
                    "parallelism": f"replicas x{world} (token data parallel, no exchange)"},
         "roofline": roof,
         "block": {"hbm_gbs": alg["block_bytes"] / block_s / 1e9,
                   "hbm_frac": alg["block_bytes"] / block_s / 1e9 / peaks["hbm_gbs"],
                   "tflops": alg["expert_flops"] / block_s / 1e12,
-                  "tensor_frac": alg["expert_flops"] / block_s / 1e12 / peaks["bf16_tflops"],
+                  "tensor_frac": alg["expert_flops"] / block_s / 1e12 / tc_peak,
+                  "tensor_frac_of_burst": alg["expert_flops"] / block_s / 1e12
+                  / peaks["bf16_tflops"],
+                  "tensor_peak_kind": "sustained" if sustained else "burst",
                   "touched_experts": alg["touched_experts"]},
-        "stages_ms": stage_mean,
+        "stages_ms": None if args.replay else stage_mean,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * wl.H * 2,
                 "d2h_bytes_per_step": wl.T * wl.H * 2},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (KERNELS_PER_STEP - (1 if args.replay else 0)) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -392,7 +412,8 @@ def run_ours(args, wl):
                                 "kind": "oracle", "sample": sample.desc, "seconds": dt}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    trace.close()
+    if trace is not None:
+        trace.close()
     if world > 1:
         dist.destroy_process_group()
     return 0
@@ -406,6 +427,10 @@ def main():
     ap.add_argument("--workload", default="decode", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bias-mode", type=int, default=0, choices=[0, 1],
+                    help="0: router bias on the logits; 1: on the choice scores only")
+    ap.add_argument("--replay", action="store_true",
+                    help="time the expert path with recorded routes (beam_moe_forward_routed)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (small profiling captures only)")
     ap.add_argument("--experts", type=int, default=None,
