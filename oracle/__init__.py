@@ -35,6 +35,20 @@ def lib():
         L.oracle_swiglu_expert.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, P, P]
         L.oracle_experts.restype = ctypes.c_int
         L.oracle_experts.argtypes = [ctypes.POINTER(OracleCfg), ctypes.c_int64, P, P, P, P, P, P]
+        L.oracle_e2m1_value.restype = ctypes.c_double
+        L.oracle_e2m1_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_value.restype = ctypes.c_double
+        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_e2m1_encode.restype = ctypes.c_uint8
+        L.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+        L.oracle_nvfp4_quantize.restype = ctypes.c_int
+        L.oracle_nvfp4_quantize.argtypes = [P, ctypes.c_int64, ctypes.c_float, P, P]
+        L.oracle_experts_nvfp4.restype = ctypes.c_int
+        L.oracle_experts_nvfp4.argtypes = [ctypes.POINTER(OracleCfg), ctypes.c_int64, P, P, P, P,
+                                           P, P, P, ctypes.c_double, ctypes.c_double,
+                                           ctypes.c_float, ctypes.c_float, P]
         _lib = L
     return _lib
 
@@ -121,3 +135,85 @@ def forward(cfg, x_bits, w_router, bias, w13_of, w2_of):
     """Route, then run the experts: returns (route dict, out [T, H] fp64)."""
     r = route(cfg, x_bits, w_router, bias)
     return r, experts(cfg, x_bits, r["ids"], r["weights"], w13_of, w2_of)
+
+
+# ------------------------------------------------------------------- NVFP4
+
+def e4m3_encode(values):
+    return np.array([lib().oracle_e4m3_encode(float(v)) for v in np.ravel(values)],
+                    dtype=np.uint8).reshape(np.shape(values))
+
+
+def e4m3_value(bytes_):
+    return np.array([lib().oracle_e4m3_value(int(b)) for b in np.ravel(bytes_)]).reshape(
+        np.shape(bytes_))
+
+
+def e2m1_encode(values):
+    return np.array([lib().oracle_e2m1_encode(float(v)) for v in np.ravel(values)],
+                    dtype=np.uint8).reshape(np.shape(values))
+
+
+def e2m1_value(codes):
+    return np.array([lib().oracle_e2m1_value(int(c)) for c in np.ravel(codes)]).reshape(
+        np.shape(codes))
+
+
+def nvfp4_quantize(values, g):
+    """Rows of fp32 values [R, K] -> (codes uint8 [R, K/2], scales uint8 [R, K/16])."""
+    v = np.ascontiguousarray(np.atleast_2d(values), dtype=np.float32)
+    R, K = v.shape
+    codes = np.zeros((R, K // 2), np.uint8)
+    sf = np.zeros((R, K // 16), np.uint8)
+    for r in range(R):
+        rc = lib().oracle_nvfp4_quantize(v[r].ctypes.data, K, g, codes[r].ctypes.data,
+                                         sf[r].ctypes.data)
+        if rc != 0:
+            raise ValueError(f"oracle_nvfp4_quantize failed ({rc})")
+    return codes, sf
+
+
+_E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def nvfp4_dequant(codes, sf, g):
+    """(codes [R, K/2], scales [R, K/16]) -> fp64 values [R, K] (table lookups only)."""
+    codes = np.atleast_2d(codes)
+    sf = np.atleast_2d(sf)
+    nib = np.stack([codes & 15, codes >> 4], axis=-1).reshape(codes.shape[0], -1)
+    v = _E2M1[nib & 7] * np.where(nib & 8, -1.0, 1.0)
+    s = e4m3_table()[sf]
+    return v * np.repeat(s, 16, axis=1) * g
+
+
+_E4M3 = None
+
+
+def e4m3_table():
+    global _E4M3
+    if _E4M3 is None:
+        _E4M3 = np.array([lib().oracle_e4m3_value(b) for b in range(256)])
+    return _E4M3
+
+
+def experts_nvfp4(cfg, x_bits, ids, weights, w13_of, w2_of, g_w13, g_w2, g_x, g_h):
+    """out [T, H] fp64 of the NVFP4 expert path; w13_of / w2_of map an expert id
+    to its (codes, scales) pair with row-major scales."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    w = np.ascontiguousarray(weights, dtype=np.float64)
+    T = x.shape[0]
+    E = cfg.n_experts
+    keep = []
+    P4 = [(ctypes.c_void_p * E)() for _ in range(4)]
+    for e in np.unique(ids):
+        arrs = [np.ascontiguousarray(a, dtype=np.uint8) for a in (*w13_of[int(e)], *w2_of[int(e)])]
+        keep += arrs
+        for j in range(4):
+            P4[j][int(e)] = arrs[j].ctypes.data
+    out = np.zeros((T, cfg.hidden))
+    rc = lib().oracle_experts_nvfp4(ctypes.byref(cfg), T, _ptr(x), _ptr(ids), _ptr(w), P4[0], P4[1],
+                                    P4[2], P4[3], g_w13, g_w2, g_x, g_h, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_experts_nvfp4 failed ({rc})")
+    return out

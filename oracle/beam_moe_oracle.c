@@ -211,3 +211,155 @@ int oracle_experts(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const in
   }
   return bad;
 }
+
+/* ------------------------------------------------------------------ NVFP4 */
+
+static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double oracle_e2m1_value(uint8_t code) {
+  double v = kE2M1[code & 7];
+  return (code & 8) ? -v : v;
+}
+
+double oracle_e4m3_value(uint8_t b) {
+  int E = (b >> 3) & 15, f = b & 7;
+  double v = E ? ldexp(1.0 + f / 8.0, E - 7) : ldexp(f / 8.0, -6);
+  return (b & 0x80) ? -v : v;
+}
+
+uint8_t oracle_e4m3_encode(float v) {
+  if (!(v > 0.0f)) return 0;
+  if (v >= 448.0f) return 0x7E;
+  int e;
+  double m = frexp((double)v, &e); /* v = m 2^e, m in [0.5, 1) */
+  if (e >= -5) {                    /* v >= 2^-6: normal */
+    double r = rint(m * 16.0);      /* 1.fff x 8, nearest, ties to even */
+    int E = e - 1 + 7;
+    if (r == 16.0) {
+      r = 8.0;
+      E += 1;
+    }
+    if (E > 15 || (E == 15 && r > 14.0)) return 0x7E;
+    return (uint8_t)((E << 3) | ((int)r - 8));
+  }
+  double r = rint(ldexp((double)v, 9)); /* subnormal: multiples of 2^-9 */
+  if (r >= 8.0) return 0x08;
+  return (uint8_t)r;
+}
+
+uint8_t oracle_e2m1_encode(float v) {
+  double a = fabs((double)v);
+  uint8_t c;
+  /* nearest grid value; at a midpoint the even code (0, 2, 4, 6) wins */
+  if (a <= 0.25) c = 0;
+  else if (a < 0.75) c = 1;
+  else if (a <= 1.25) c = 2;
+  else if (a < 1.75) c = 3;
+  else if (a <= 2.5) c = 4;
+  else if (a < 3.5) c = 5;
+  else if (a <= 5.0) c = 6;
+  else c = 7;
+  return (uint8_t)(c | (v < 0.0f ? 8u : 0u));
+}
+
+int oracle_nvfp4_quantize(const float* v, int64_t K, float g, uint8_t* codes, uint8_t* sf) {
+  if (!v || !codes || !sf || K <= 0 || K % 16 != 0 || !(g > 0.0f)) return -1;
+  for (int64_t b = 0; b < K / 16; ++b) {
+    const float* vb = v + b * 16;
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(vb[i]));
+    const float sd = amax / (6.0f * g);
+    const uint8_t s8 = oracle_e4m3_encode(sd);
+    const float d = (float)oracle_e4m3_value(s8) * g;
+    sf[b] = s8;
+    for (int i = 0; i < 16; i += 2) {
+      uint8_t lo = s8 ? oracle_e2m1_encode(vb[i] / d) : 0;
+      uint8_t hi = s8 ? oracle_e2m1_encode(vb[i + 1] / d) : 0;
+      codes[(b * 16 + i) / 2] = (uint8_t)(lo | (hi << 4));
+    }
+  }
+  return 0;
+}
+
+double oracle_nvfp4_value(const uint8_t* codes, const uint8_t* sf, int64_t i, double g) {
+  uint8_t byte = codes[i / 2];
+  uint8_t code = (i & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+  return oracle_e2m1_value(code) * oracle_e4m3_value(sf[i / 16]) * g;
+}
+
+int oracle_experts_nvfp4(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const int32_t* ids,
+                         const double* weights, const uint8_t* const* w13_codes,
+                         const uint8_t* const* w13_sf, const uint8_t* const* w2_codes,
+                         const uint8_t* const* w2_sf, double g_w13, double g_w2, float g_x,
+                         float g_h, double* out) {
+  if (!cfg_ok(cfg) || T < 0) return -1;
+  if (T == 0) return 0;
+  if (!x || !ids || !weights || !w13_codes || !w13_sf || !w2_codes || !w2_sf || !out) return -1;
+  const int H = cfg->hidden, I = cfg->inter, E = cfg->n_experts, K = cfg->top_k;
+  if (H % 16 || I % 16) return -1;
+  int bad = 0;
+#pragma omp parallel
+  {
+    float* xf = (float*)malloc(sizeof(float) * (size_t)H);
+    double* xd = (double*)malloc(sizeof(double) * (size_t)H);
+    uint8_t* xc = (uint8_t*)malloc((size_t)H / 2);
+    uint8_t* xs = (uint8_t*)malloc((size_t)H / 16);
+    float* af = (float*)malloc(sizeof(float) * (size_t)I);
+    double* ad = (double*)malloc(sizeof(double) * (size_t)I);
+    uint8_t* ac = (uint8_t*)malloc((size_t)I / 2);
+    uint8_t* as = (uint8_t*)malloc((size_t)I / 16);
+    if (!xf || !xd || !xc || !xs || !af || !ad || !ac || !as) {
+#pragma omp atomic write
+      bad = -2;
+    } else {
+#pragma omp for schedule(dynamic, 1)
+      for (int64_t t = 0; t < T; ++t) {
+        double* ot = out + t * (int64_t)H;
+        for (int h = 0; h < H; ++h) {
+          xf[h] = (float)bf16_to_double(x[t * (int64_t)H + h]);
+          ot[h] = 0.0;
+        }
+        oracle_nvfp4_quantize(xf, H, g_x, xc, xs);
+        for (int h = 0; h < H; ++h) xd[h] = oracle_nvfp4_value(xc, xs, h, (double)g_x);
+        for (int k = 0; k < K; ++k) {
+          const int e = ids[t * K + k];
+          if (e < 0 || e >= E || !w13_codes[e] || !w13_sf[e] || !w2_codes[e] || !w2_sf[e]) {
+#pragma omp atomic write
+            bad = -3;
+            continue;
+          }
+          for (int i = 0; i < I; ++i) {
+            const uint8_t* gc = w13_codes[e] + (int64_t)i * (H / 2);
+            const uint8_t* gs = w13_sf[e] + (int64_t)i * (H / 16);
+            const uint8_t* uc = w13_codes[e] + (int64_t)(I + i) * (H / 2);
+            const uint8_t* us = w13_sf[e] + (int64_t)(I + i) * (H / 16);
+            double g = 0.0, u = 0.0;
+            for (int h = 0; h < H; ++h) {
+              g += oracle_nvfp4_value(gc, gs, h, g_w13) * xd[h];
+              u += oracle_nvfp4_value(uc, us, h, g_w13) * xd[h];
+            }
+            af[i] = (float)(g / (1.0 + exp(-g)) * u); /* silu(g) * u, then fp32 */
+          }
+          oracle_nvfp4_quantize(af, I, g_h, ac, as);
+          for (int i = 0; i < I; ++i) ad[i] = oracle_nvfp4_value(ac, as, i, (double)g_h);
+          for (int j = 0; j < H; ++j) {
+            const uint8_t* dc = w2_codes[e] + (int64_t)j * (I / 2);
+            const uint8_t* ds = w2_sf[e] + (int64_t)j * (I / 16);
+            double acc = 0.0;
+            for (int i = 0; i < I; ++i) acc += oracle_nvfp4_value(dc, ds, i, g_w2) * ad[i];
+            ot[j] += weights[t * K + k] * acc;
+          }
+        }
+      }
+    }
+    free(xf);
+    free(xd);
+    free(xc);
+    free(xs);
+    free(af);
+    free(ad);
+    free(ac);
+    free(as);
+  }
+  return bad;
+}

@@ -83,6 +83,46 @@ int oracle_experts(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const in
                    const double* weights, const uint16_t* const* w13, const uint16_t* const* w2,
                    double* out);
 
+/* ------------------------------------------------------------------ NVFP4
+ * The 4-bit format the launch post names for Blackwell deployment ("Welcome
+ * Beam", section "Mixture of Experts": the NVFP4 checkpoint stores most
+ * parameters in 4-bit precision for NVIDIA Blackwell GPUs): E2M1 values
+ * {0, .5, 1, 1.5, 2, 3, 4, 6} with a sign bit, one FP8 E4M3 scale per 16
+ * consecutive elements along the contraction dimension, one FP32 scale per
+ * tensor. value = e2m1(code) * e4m3(scale) * tensor_scale. Codes are packed
+ * two per byte, element 2j in the low nibble.
+ */
+double oracle_e2m1_value(uint8_t code);  /* low 4 bits used */
+double oracle_e4m3_value(uint8_t byte);
+/* Round to nearest, ties to even, saturating at 448 (v >= 0 finite). */
+uint8_t oracle_e4m3_encode(float v);
+/* Round to nearest, ties to even, saturating at +-6. */
+uint8_t oracle_e2m1_encode(float v);
+
+/* Quantise K values (K a multiple of 16), every step in fp32: per block,
+ * amax = max |v|, scale = e4m3(amax / (6 g)), then each code =
+ * e2m1(v / (scale * g)) (all zero when the scale is zero). codes[K/2],
+ * sf[K/16]. */
+int oracle_nvfp4_quantize(const float* v, int64_t K, float g, uint8_t* codes, uint8_t* sf);
+
+/* Dequantised value of element i of a packed row. */
+double oracle_nvfp4_value(const uint8_t* codes, const uint8_t* sf, int64_t i, double g);
+
+/*
+ * Expert path with NVFP4 experts and NVFP4 activations (the W4A4 scheme the
+ * vLLM recipe's FlashInfer TRT-LLM backend uses): each token's x (bf16) is
+ * quantised with tensor scale g_x; g = Wg xq, u = Wu xq exactly in fp64 on the
+ * dequantised values; a = silu(g) * u in fp64, rounded to fp32 and quantised
+ * with g_h; y = Wd aq; out[t] = sum_k weights[t][k] y.
+ * w13_codes[e] [2I][H/2], w13_sf[e] [2I][H/16], w2_codes[e] [H][I/2],
+ * w2_sf[e] [H][I/16] (scales row-major).
+ */
+int oracle_experts_nvfp4(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const int32_t* ids,
+                         const double* weights, const uint8_t* const* w13_codes,
+                         const uint8_t* const* w13_sf, const uint8_t* const* w2_codes,
+                         const uint8_t* const* w2_sf, double g_w13, double g_w2, float g_x,
+                         float g_h, double* out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -113,6 +113,8 @@ def host_lib():
                                           ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32,
                                           ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                                           ctypes.c_int64]
+        lib.synth_host_nvfp4.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                         ctypes.c_int64, ctypes.c_int64, ctypes.c_uint64]
         lib.synth_host_pick.restype = ctypes.c_int
         lib.synth_host_pick.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64,
                                         ctypes.c_void_p]
@@ -135,6 +137,9 @@ def cuda_lib():
         lib.synth_dev_x.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                     ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32,
                                     ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]
+        lib.synth_dev_nvfp4.restype = ctypes.c_int
+        lib.synth_dev_nvfp4.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                        ctypes.c_int64, ctypes.c_uint64, ctypes.c_void_p]
         _cuda = lib
     return _cuda
 
@@ -262,6 +267,55 @@ def dev_w13(wl, ptr, stream, seed=SEED):
 
 def dev_w2(wl, ptr, stream, seed=SEED):
     dev_normal_bf16(ptr, wl.w2_elems, STREAM_W2, stream, sigma=wl.sigma_w, seed=seed)
+
+
+# ------------------------------------------------------------------- NVFP4
+
+# Per-tensor FP32 scales of the synthetic NVFP4 experts (weights) and the
+# static activation scales used when the forward quantises x and h.
+NVFP4_WEIGHT_SCALE = 2.0 ** -7
+NVFP4_ACT_SCALE = 2.0 ** -6
+
+
+def host_nvfp4_rows(stream, r0, n, K, seed=SEED):
+    """(codes uint8 [n, K/2], scales uint8 [n, K/16]) of rows r0 .. r0+n-1."""
+    codes = np.empty((n, K // 2), dtype=np.uint8)
+    sf = np.empty((n, K // 16), dtype=np.uint8)
+    host_lib().synth_host_nvfp4(codes.ctypes.data, sf.ctypes.data, r0, n, K,
+                                _u64(key(stream, seed)))
+    return codes, sf
+
+
+def host_expert_w13_nvfp4(wl, e, seed=SEED):
+    """NVFP4 gate/up weights of expert e: codes [2I, H/2], scales [2I, H/16]."""
+    return host_nvfp4_rows(STREAM_W13, e * 2 * wl.I, 2 * wl.I, wl.H, seed)
+
+
+def host_expert_w2_nvfp4(wl, e, seed=SEED):
+    """NVFP4 down weights of expert e: codes [H, I/2], scales [H, I/16]."""
+    return host_nvfp4_rows(STREAM_W2, e * wl.H, wl.H, wl.I, seed)
+
+
+def dev_nvfp4(stream_id, codes_ptr, sf_ptr, rows, K, stream, seed=SEED):
+    """Device NVFP4 matrix [rows][K]: codes and scales in the MMA scale layout."""
+    _check(cuda_lib().synth_dev_nvfp4(codes_ptr, sf_ptr, rows, K, _u64(key(stream_id, seed)),
+                                      stream), "nvfp4")
+
+
+def dev_w13_nvfp4(wl, codes_ptr, sf_ptr, stream, seed=SEED):
+    dev_nvfp4(STREAM_W13, codes_ptr, sf_ptr, wl.E * 2 * wl.I, wl.H, stream, seed)
+
+
+def dev_w2_nvfp4(wl, codes_ptr, sf_ptr, stream, seed=SEED):
+    dev_nvfp4(STREAM_W2, codes_ptr, sf_ptr, wl.E * wl.H, wl.I, stream, seed)
+
+
+def sf_offset(r, b, K):
+    """Byte offset of (row, 16-block) in the block-scaled MMA scale layout."""
+    r = np.asarray(r, dtype=np.int64)
+    b = np.asarray(b, dtype=np.int64)
+    rr = r % 128
+    return ((r // 128) * (K // 64) + b // 4) * 512 + (rr % 32) * 16 + (rr // 32) * 4 + (b % 4)
 
 
 def bf16_to_f32(bits):

@@ -93,4 +93,52 @@ SYNTH_HD uint16_t synth_bf16_bits(float f) {
   return (uint16_t)(u >> 16);
 }
 
+/* ------------------------------------------------------------------ NVFP4
+ * Synthetic NVFP4 expert weights (4-bit E2M1 values, one FP8 E4M3 scale per
+ * 16 consecutive elements of a row, one FP32 scale per tensor), drawn
+ * directly in the format: no quantisation arithmetic is involved.
+ *  - element code: a standard-normal deviate z, times 2, mapped to the nearest
+ *    E2M1 magnitude {0, .5, 1, 1.5, 2, 3, 4, 6} (fixed thresholds; z is a
+ *    multiple of 2^-17 so no tie can occur), sign bit 3;
+ *  - block scale: E4M3 byte 0x38 + (u mod 8), i.e. 1.0 .. 1.875.
+ * With a tensor scale of 2^-7 the values have a standard deviation of about
+ * 0.02, like the bf16 experts. */
+SYNTH_HD uint8_t synth_e2m1_code(float z) {
+  float m = fabsf(z) * 2.0f;
+  uint8_t c;
+  if (m < 0.25f) c = 0;
+  else if (m < 0.75f) c = 1;
+  else if (m < 1.25f) c = 2;
+  else if (m < 1.75f) c = 3;
+  else if (m < 2.5f) c = 4;
+  else if (m < 3.5f) c = 5;
+  else if (m < 5.0f) c = 6;
+  else c = 7;
+  return (uint8_t)(c | (z < 0.0f && c != 0 ? 8u : 0u));
+}
+
+/* Packed byte j of a weight row: elements 2j (low nibble) and 2j + 1. The
+ * element index of the row's first element is `idx_row`. */
+SYNTH_HD uint8_t synth_nvfp4_byte(uint64_t key, uint64_t idx_row, uint64_t j) {
+  uint8_t lo = synth_e2m1_code(synth_z(key, idx_row + 2 * j));
+  uint8_t hi = synth_e2m1_code(synth_z(key, idx_row + 2 * j + 1));
+  return (uint8_t)(lo | (hi << 4));
+}
+
+/* E4M3 scale byte of the 16-element block `blk` (global block index). */
+SYNTH_HD uint8_t synth_nvfp4_scale(uint64_t key, uint64_t blk) {
+  return (uint8_t)(0x38u + (uint32_t)(synth_u64(key ^ 0x5CA1Eull, blk) & 7u));
+}
+
+/* Byte offset, inside a scale array in the block-scaled MMA layout, of the
+ * scale of row r, 16-element block b, for a matrix whose rows hold K
+ * elements: 512-byte atoms of 128 rows x 4 blocks, atoms ordered (row block,
+ * 64-element chunk) with the chunk fastest; inside an atom, row r0 + 32 r1
+ * and block kb sit at byte 16 r0 + 4 r1 + kb. */
+SYNTH_HD uint64_t synth_sf_offset(uint64_t r, uint64_t b, uint64_t K) {
+  uint64_t atom = (r / 128) * (K / 64) + b / 4;
+  uint64_t rr = r % 128;
+  return atom * 512 + (rr % 32) * 16 + (rr / 32) * 4 + (b % 4);
+}
+
 #endif /* BEAM_SYNTH_H */

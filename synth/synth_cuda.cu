@@ -40,6 +40,24 @@ __global__ void fill_x(uint16_t* x, int64_t T, int64_t H, uint64_t key_x, uint64
   }
 }
 
+__global__ void fill_nvfp4_codes(uint8_t* codes, int64_t rows, int64_t K, uint64_t key) {
+  const int64_t n = rows * (K / 2);
+  int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const int64_t r = i / (K / 2), j = i - r * (K / 2);
+    codes[i] = synth_nvfp4_byte(key, (uint64_t)r * (uint64_t)K, (uint64_t)j);
+  }
+}
+
+__global__ void fill_nvfp4_scales(uint8_t* sf, int64_t rows, int64_t K, uint64_t key) {
+  const int64_t n = rows * (K / 16);
+  int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const int64_t r = i / (K / 16), b = i - r * (K / 16);
+    sf[synth_sf_offset((uint64_t)r, (uint64_t)b, (uint64_t)K)] = synth_nvfp4_scale(key, (uint64_t)i);
+  }
+}
+
 int grid_for(int64_t n) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -76,6 +94,17 @@ int synth_dev_x(void* x, int64_t T, int64_t H, uint64_t key_x, uint64_t key_c, i
   if (T * H <= 0) return 0;
   fill_x<<<grid_for(T * H), 256, 0, (cudaStream_t)stream>>>(
       (uint16_t*)x, T, H, key_x, key_c, n_centres, sigma, (const int32_t*)attempts);
+  return (int)cudaGetLastError();
+}
+
+/* NVFP4 weights of a whole [rows][K] matrix (rows a multiple of 128): packed
+ * codes [rows][K/2] and scales in the block-scaled MMA layout. */
+int synth_dev_nvfp4(void* codes, void* sf, int64_t rows, int64_t K, uint64_t key, void* stream) {
+  if (rows * K <= 0) return 0;
+  fill_nvfp4_codes<<<grid_for(rows * K / 2), 256, 0, (cudaStream_t)stream>>>((uint8_t*)codes, rows,
+                                                                             K, key);
+  fill_nvfp4_scales<<<grid_for(rows * K / 16), 256, 0, (cudaStream_t)stream>>>((uint8_t*)sf, rows,
+                                                                               K, key);
   return (int)cudaGetLastError();
 }
 

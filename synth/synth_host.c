@@ -87,3 +87,17 @@ int synth_host_pick(uint64_t key, int64_t n, int64_t k, int64_t* out) {
   qsort(out, (size_t)k, sizeof(int64_t), synth_index_cmp);
   return 0;
 }
+
+/* NVFP4 weights of rows [r0, r0 + n) of a matrix with K elements per row:
+ * packed codes [n][K/2] and the E4M3 scales row-major [n][K/16] (the device
+ * fill writes the same scales in the block-scaled MMA layout instead). */
+void synth_host_nvfp4(uint8_t* codes, uint8_t* sf, int64_t r0, int64_t n, int64_t K,
+                      uint64_t key) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = r0; r < r0 + n; ++r) {
+    for (int64_t j = 0; j < K / 2; ++j)
+      codes[(r - r0) * (K / 2) + j] = synth_nvfp4_byte(key, (uint64_t)r * (uint64_t)K, (uint64_t)j);
+    for (int64_t b = 0; b < K / 16; ++b)
+      sf[(r - r0) * (K / 16) + b] = synth_nvfp4_scale(key, (uint64_t)r * (uint64_t)(K / 16) + (uint64_t)b);
+  }
+}
