@@ -74,8 +74,9 @@ typedef enum beam_moe_status {
 } beam_moe_status;
 
 typedef enum beam_moe_op {
-  BEAM_MOE_OP_ROUTE = 0,   /* beam_moe_route                            */
-  BEAM_MOE_OP_FORWARD = 1, /* beam_moe_forward, beam_moe_forward_routed */
+  BEAM_MOE_OP_ROUTE = 0,         /* beam_moe_route                            */
+  BEAM_MOE_OP_FORWARD = 1,       /* beam_moe_forward, beam_moe_forward_routed */
+  BEAM_MOE_OP_FORWARD_NVFP4 = 2, /* beam_moe_forward_nvfp4                    */
 } beam_moe_op;
 
 /* Bytes of workspace the operation needs for T tokens (a pure host function). */
@@ -165,6 +166,56 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_routed(const beam_moe_cfg* cfg, in
                                         void* stream);
 
 /*
+ * NVFP4 experts ("Welcome Beam", section "Mixture of Experts": the NVFP4
+ * checkpoint stores most parameters in 4-bit precision for NVIDIA Blackwell
+ * GPUs). A value is e2m1(code) * e4m3(scale) * tensor_scale: 4-bit E2M1 codes
+ * {0, .5, 1, 1.5, 2, 3, 4, 6} with a sign bit, packed two per byte (element
+ * 2j in the low nibble), one FP8 E4M3 scale per 16 consecutive elements of a
+ * row, one FP32 scale per tensor. Scales are stored in the block-scaled MMA
+ * layout: for a matrix with K elements per row, the scale of row r and
+ * 16-element block b is at byte
+ *   ((r / 128) * (K / 64) + b / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + b % 4.
+ * All pointers are device memory, 16-byte aligned.
+ */
+typedef struct beam_moe_nvfp4_experts {
+  const uint8_t* w13_codes;  /* [E][2I][H/2]: rows 0..I-1 gate, I..2I-1 up   */
+  const uint8_t* w13_scales; /* E * 2I * H / 16 bytes, layout above (K = H)  */
+  const uint8_t* w2_codes;   /* [E][H][I/2]                                  */
+  const uint8_t* w2_scales;  /* E * H * I / 16 bytes, layout above (K = I)   */
+  float w13_scale;           /* tensor scale of W13                          */
+  float w2_scale;            /* tensor scale of W2                           */
+  float x_scale;             /* tensor scale x is quantised with             */
+  float h_scale;             /* tensor scale h = silu(g) * u is quantised with */
+} beam_moe_nvfp4_experts;
+
+/*
+ * Whole block with NVFP4 experts and NVFP4 activations (W4A4, the scheme of
+ * the vLLM recipe's FlashInfer TRT-LLM NVFP4 backend): routing as
+ * beam_moe_forward; every token's x is quantised per 16 elements (scale =
+ * e4m3(amax / (6 x_scale)), code = e2m1(x / (scale x_scale)), round to
+ * nearest even, saturating); g, u = W13 x on block-scaled FP4 tensor cores
+ * with FP32 accumulation; h = silu(g) * u in FP32, quantised the same way with
+ * h_scale; y = W2 h in FP32; out as beam_moe_forward. Requires hidden and
+ * inter to be multiples of 256. Workspace: BEAM_MOE_OP_FORWARD_NVFP4.
+ */
+BEAM_MOE_API beam_moe_status beam_moe_forward_nvfp4(const beam_moe_cfg* cfg, int64_t T,
+                                                    const uint16_t* x, const float* w_router,
+                                                    const float* bias,
+                                                    const beam_moe_nvfp4_experts* experts,
+                                                    uint16_t* out, int32_t* topk_ids,
+                                                    float* topk_w, int32_t* expert_counts,
+                                                    void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Quantise `rows` rows of K fp32 values (device, K a multiple of 16) to
+ * NVFP4 with tensor scale g, as beam_moe_forward_nvfp4 quantises x and h:
+ * codes [rows][K/2] and scales row-major [rows][K/16] (device outputs).
+ */
+BEAM_MOE_API beam_moe_status beam_moe_nvfp4_quantize(int64_t rows, int64_t K, const float* v,
+                                                     float g, uint8_t* codes, uint8_t* scales,
+                                                     void* stream);
+
+/*
  * Stage timing. A trace records CUDA events around each stage of the calls
  * it is passed to: slot i of stage s is the time of that stage in the i-th
  * traced call since the last reset. Stages: 0 router GEMM, 1 top-k and
@@ -178,6 +229,11 @@ BEAM_MOE_API beam_moe_status beam_moe_trace_destroy(beam_moe_trace* trace);
 BEAM_MOE_API beam_moe_status beam_moe_trace_reset(beam_moe_trace* trace);
 /* ms[i * BEAM_MOE_N_STAGES + s] for i < *n_calls (at most capacity). */
 BEAM_MOE_API beam_moe_status beam_moe_trace_read(beam_moe_trace* trace, float* ms, int32_t* n_calls);
+BEAM_MOE_API beam_moe_status beam_moe_forward_nvfp4_traced(
+    const beam_moe_cfg* cfg, int64_t T, const uint16_t* x, const float* w_router,
+    const float* bias, const beam_moe_nvfp4_experts* experts, uint16_t* out, int32_t* topk_ids,
+    float* topk_w, int32_t* expert_counts, void* ws, size_t ws_bytes, void* stream,
+    beam_moe_trace* trace);
 BEAM_MOE_API beam_moe_status beam_moe_forward_traced(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
                                         const float* w_router, const float* bias,
                                         const uint16_t* w13, const uint16_t* w2, uint16_t* out,

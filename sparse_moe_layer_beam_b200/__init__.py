@@ -16,7 +16,8 @@ import os
 
 __all__ = ["BeamMoeCfg", "BeamMoeError", "Trace", "OP_ROUTE", "OP_FORWARD", "N_STAGES",
            "STAGE_NAMES", "lib", "beam_cfg", "beam_moe_workspace_size", "beam_moe_route",
-           "beam_moe_route_noalloc",
+           "beam_moe_route_noalloc", "BeamMoeNvfp4Experts", "OP_FORWARD_NVFP4", "nvfp4_experts",
+           "beam_moe_forward_nvfp4", "beam_moe_nvfp4_quantize",
            "beam_moe_forward", "beam_moe_forward_routed", "beam_moe_forward_traced",
            "beam_moe_check"]
 
@@ -25,6 +26,7 @@ LIB_PATH = os.path.join(_HERE, "libbeam_moe.so")
 
 OP_ROUTE = 0
 OP_FORWARD = 1
+OP_FORWARD_NVFP4 = 2
 N_STAGES = 7
 STAGE_NAMES = ("router_gemm", "router_topk", "scan", "permute", "gateup_gemm", "down_gemm",
                "combine")
@@ -36,6 +38,14 @@ class BeamMoeCfg(ctypes.Structure):
                 ("topk_group", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("renormalize", ctypes.c_int32), ("bias_mode", ctypes.c_int32),
                 ("routed_scale", ctypes.c_float)]
+
+
+class BeamMoeNvfp4Experts(ctypes.Structure):
+    """NVFP4 expert weights (device pointers) and tensor scales."""
+    _fields_ = [("w13_codes", ctypes.c_void_p), ("w13_scales", ctypes.c_void_p),
+                ("w2_codes", ctypes.c_void_p), ("w2_scales", ctypes.c_void_p),
+                ("w13_scale", ctypes.c_float), ("w2_scale", ctypes.c_float),
+                ("x_scale", ctypes.c_float), ("h_scale", ctypes.c_float)]
 
 
 class BeamMoeError(RuntimeError):
@@ -57,6 +67,13 @@ _SIGS = {
                                 ctypes.c_size_t, _P],
     "beam_moe_forward_traced": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                 ctypes.c_size_t, _P, _P],
+    "beam_moe_forward_nvfp4": [_CFG, ctypes.c_int64, _P, _P, _P,
+                               ctypes.POINTER(BeamMoeNvfp4Experts), _P, _P, _P, _P, _P,
+                               ctypes.c_size_t, _P],
+    "beam_moe_forward_nvfp4_traced": [_CFG, ctypes.c_int64, _P, _P, _P,
+                                      ctypes.POINTER(BeamMoeNvfp4Experts), _P, _P, _P, _P, _P,
+                                      ctypes.c_size_t, _P, _P],
+    "beam_moe_nvfp4_quantize": [ctypes.c_int64, ctypes.c_int64, _P, ctypes.c_float, _P, _P, _P],
     "beam_moe_trace_create": [ctypes.c_int32, ctypes.POINTER(_P)],
     "beam_moe_trace_destroy": [_P],
     "beam_moe_trace_reset": [_P],
@@ -157,6 +174,31 @@ def beam_moe_forward_routed(cfg, x, topk_ids, topk_w, w13, w2, out, ws, expert_c
                                          _ptr(expert_counts), _ptr(ws),
                                          ws.numel() * ws.element_size(), _stream(stream)),
            "beam_moe_forward_routed")
+
+
+def nvfp4_experts(w13_codes, w13_scales, w2_codes, w2_scales, w13_scale, w2_scale, x_scale,
+                  h_scale):
+    return BeamMoeNvfp4Experts(_ptr(w13_codes), _ptr(w13_scales), _ptr(w2_codes),
+                               _ptr(w2_scales), w13_scale, w2_scale, x_scale, h_scale)
+
+
+def beam_moe_forward_nvfp4(cfg, x, w_router, bias, experts, out, ws, topk_ids=None, topk_w=None,
+                           expert_counts=None, stream=None, trace=None):
+    T = x.shape[0]
+    args = (ctypes.byref(cfg), T, _ptr(x), _ptr(w_router), _ptr(bias), ctypes.byref(experts),
+            _ptr(out), _ptr(topk_ids), _ptr(topk_w), _ptr(expert_counts), _ptr(ws),
+            ws.numel() * ws.element_size(), _stream(stream))
+    if trace is None:
+        _check(lib().beam_moe_forward_nvfp4(*args), "beam_moe_forward_nvfp4")
+    else:
+        _check(lib().beam_moe_forward_nvfp4_traced(*args, trace.handle),
+               "beam_moe_forward_nvfp4_traced")
+
+
+def beam_moe_nvfp4_quantize(v, g, codes, scales, stream=None):
+    rows, K = v.shape
+    _check(lib().beam_moe_nvfp4_quantize(rows, K, _ptr(v), g, _ptr(codes), _ptr(scales),
+                                         _stream(stream)), "beam_moe_nvfp4_quantize")
 
 
 def beam_moe_check(ws, stream=None):

@@ -124,6 +124,21 @@ cudaError_t encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t col
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 2-D byte tensor [rows][cols], box {box_cols, box_rows}, 128-byte swizzle.
+cudaError_t encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                              uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // W13 [E][2I][H] seen as 5-D {H, 16, 2, I/16, E} (k, row in a 16-row block,
 // gate/up, block, expert): a box {64, 16, 2, 4, 1} lands in shared memory as
 // 128 rows ordered gate 0-15, up 0-15, gate 16-31, up 16-31, ... of 64
@@ -297,22 +312,106 @@ beam_moe_status forward_impl(const beam_moe_cfg* cfg, int64_t T, const uint16_t*
   return BEAM_MOE_OK;
 }
 
+bool positive_finite(float v) { return isfinite(v) && v > 0.0f; }
+
+beam_moe_status forward_nvfp4_impl(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                                   const float* w_router, const float* bias,
+                                   const beam_moe_nvfp4_experts* ex, uint16_t* out,
+                                   int32_t* topk_ids, float* topk_w, int32_t* expert_counts,
+                                   void* ws, size_t ws_bytes, void* stream,
+                                   beam_moe_trace* trace) {
+  BEAM_TRY(common_checks(cfg, T, ws, ws_bytes, BEAM_MOE_OP_FORWARD_NVFP4));
+  if (T == 0) return BEAM_MOE_OK;
+  if (!ex) return BEAM_MOE_ERR_INVALID_ARG;
+  BEAM_TRY(check_ptrs({x, w_router, ex->w13_codes, ex->w13_scales, ex->w2_codes, ex->w2_scales,
+                       out},
+                      {bias, topk_ids, topk_w, expert_counts}));
+  if (!positive_finite(ex->w13_scale) || !positive_finite(ex->w2_scale) ||
+      !positive_finite(ex->x_scale) || !positive_finite(ex->h_scale))
+    return BEAM_MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
+  const beam::Fp4Layout F = beam::make_layout_nvfp4(*cfg, T, beam::device_sm_count());
+  const Layout& L = F.base;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  Recorder rec(trace, st);
+  BEAM_CUDA(cudaMemsetAsync(w + L.status, 0, 256, st));
+  BEAM_CUDA(rec.mark(0));
+  BEAM_CUDA(beam::launch_router_logits(*cfg, L, x, w_router, w, st));
+  BEAM_CUDA(rec.mark(1));
+  BEAM_CUDA(beam::launch_router_topk(*cfg, L, bias, w, st));
+  BEAM_CUDA(rec.mark(2));
+  BEAM_CUDA(beam::launch_scan(*cfg, L, w, expert_counts, st));
+  BEAM_CUDA(rec.mark(3));
+  BEAM_CUDA(beam::launch_permute_nvfp4(*cfg, F, x, ex->x_scale, w, st));
+  BEAM_CUDA(rec.mark(4));
+  BEAM_CUDA(beam::launch_gateup_nvfp4(*cfg, F, *ex, w, st));
+  BEAM_CUDA(rec.mark(5));
+  BEAM_CUDA(beam::launch_down_nvfp4(*cfg, F, *ex, w, st));
+  BEAM_CUDA(rec.mark(6));
+  BEAM_CUDA(beam::launch_combine(*cfg, L, out, w, st));
+  BEAM_CUDA(rec.mark(7));
+  BEAM_CUDA(beam::launch_copy_routes(*cfg, L, topk_ids, topk_w, w, st));
+  rec.done();
+  return BEAM_MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+beam_moe_status beam_moe_forward_nvfp4(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                                       const float* w_router, const float* bias,
+                                       const beam_moe_nvfp4_experts* experts, uint16_t* out,
+                                       int32_t* topk_ids, float* topk_w, int32_t* expert_counts,
+                                       void* ws, size_t ws_bytes, void* stream) {
+  return forward_nvfp4_impl(cfg, T, x, w_router, bias, experts, out, topk_ids, topk_w,
+                            expert_counts, ws, ws_bytes, stream, nullptr);
+}
+
+beam_moe_status beam_moe_forward_nvfp4_traced(const beam_moe_cfg* cfg, int64_t T,
+                                              const uint16_t* x, const float* w_router,
+                                              const float* bias,
+                                              const beam_moe_nvfp4_experts* experts,
+                                              uint16_t* out, int32_t* topk_ids, float* topk_w,
+                                              int32_t* expert_counts, void* ws, size_t ws_bytes,
+                                              void* stream, beam_moe_trace* trace) {
+  if (!trace) return BEAM_MOE_ERR_INVALID_ARG;
+  return forward_nvfp4_impl(cfg, T, x, w_router, bias, experts, out, topk_ids, topk_w,
+                            expert_counts, ws, ws_bytes, stream, trace);
+}
+
+beam_moe_status beam_moe_nvfp4_quantize(int64_t rows, int64_t K, const float* v, float g,
+                                        uint8_t* codes, uint8_t* scales, void* stream) {
+  if (rows < 0 || K <= 0 || K % 16 != 0 || !positive_finite(g)) return BEAM_MOE_ERR_INVALID_ARG;
+  if (rows == 0) return BEAM_MOE_OK;
+  if (!v || !codes || !scales) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!aligned16(v) || !aligned16(codes) || !aligned16(scales)) return BEAM_MOE_ERR_ALIGNMENT;
+  BEAM_CUDA(beam::launch_quantize_rows(rows, K, v, g, codes, scales,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+  return BEAM_MOE_OK;
+}
 
 beam_moe_status beam_moe_workspace_size(const beam_moe_cfg* cfg, int64_t T, beam_moe_op op,
                                         size_t* bytes) {
   BEAM_TRY(check_cfg(cfg));
   BEAM_TRY(check_T(cfg, T));
-  if (!bytes || (op != BEAM_MOE_OP_ROUTE && op != BEAM_MOE_OP_FORWARD))
+  if (!bytes || (op != BEAM_MOE_OP_ROUTE && op != BEAM_MOE_OP_FORWARD &&
+                 op != BEAM_MOE_OP_FORWARD_NVFP4))
     return BEAM_MOE_ERR_INVALID_ARG;
+  if (op == BEAM_MOE_OP_FORWARD_NVFP4 && !beam::nvfp4_supported(*cfg))
+    return BEAM_MOE_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) {
     *bytes = 0;
     return BEAM_MOE_OK;
   }
   // Sized for the largest split-K any device could pick (148 SMs bound it for
   // B200; the 1024-SM bound keeps the size valid on any part).
+  if (op == BEAM_MOE_OP_FORWARD_NVFP4) {
+    *bytes = beam::make_layout_nvfp4(*cfg, T, 1024).base.total;
+    return BEAM_MOE_OK;
+  }
   Layout L = beam::make_layout(*cfg, T, 1024);
   *bytes = op == BEAM_MOE_OP_ROUTE ? L.route_end : L.total;
   return BEAM_MOE_OK;

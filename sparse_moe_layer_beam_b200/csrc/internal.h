@@ -52,6 +52,19 @@ struct Layout {
 
 Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms);
 
+// NVFP4 path: the routing layout (token tiles of 128 rows, expert segments
+// padded to them) plus quantised activations and their scales.
+struct Fp4Layout {
+  Layout base;    // routing arrays; base.xp holds the fp32 down output y
+  int64_t rows;   // bound on the padded rows
+  size_t xq;      // uint8[rows * H/2] quantised x, expert segments 128-row aligned
+  size_t xsf;     // uint8[rows * H/16] their scales (atom layout)
+  size_t hq;      // uint8[rows * I/2] quantised h
+  size_t hsf;     // uint8[rows * I/16]
+};
+Fp4Layout make_layout_nvfp4(const beam_moe_cfg& c, int64_t T, int sms);
+bool nvfp4_supported(const beam_moe_cfg& c);
+
 // ---- launchers (each enqueues on `st`, returns cudaGetLastError()) --------
 cudaError_t launch_router_logits(const beam_moe_cfg& c, const Layout& L, const uint16_t* x,
                                  const float* w_router, char* ws, cudaStream_t st);
@@ -83,6 +96,17 @@ cudaError_t encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t col
 
 cudaError_t encode_tmap_w13_interleaved(CUtensorMap* map, const void* w13, uint64_t H, uint64_t I,
                                         uint64_t E);
+
+cudaError_t encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                              uint32_t box_cols, uint32_t box_rows);
+cudaError_t launch_permute_nvfp4(const beam_moe_cfg& c, const Fp4Layout& F, const uint16_t* x,
+                                 float gx, char* ws, cudaStream_t st);
+cudaError_t launch_gateup_nvfp4(const beam_moe_cfg& c, const Fp4Layout& F,
+                                const beam_moe_nvfp4_experts& w, char* ws, cudaStream_t st);
+cudaError_t launch_down_nvfp4(const beam_moe_cfg& c, const Fp4Layout& F,
+                              const beam_moe_nvfp4_experts& w, char* ws, cudaStream_t st);
+cudaError_t launch_quantize_rows(int64_t rows, int64_t K, const float* v, float g, uint8_t* codes,
+                                 uint8_t* sf, cudaStream_t st);
 
 int device_sm_count();
 

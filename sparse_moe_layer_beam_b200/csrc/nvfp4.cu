@@ -1,0 +1,550 @@
+// nvfp4.cu - the Beam MoE block with NVFP4 experts and NVFP4 activations
+// (W4A4): the 4-bit format the launch post "Welcome Beam" names for Blackwell
+// deployment (section "Mixture of Experts": the NVFP4 checkpoint stores most
+// parameters in 4-bit precision for NVIDIA Blackwell GPUs), with E2M1 values,
+// one FP8 E4M3 scale per 16 elements along K and one FP32 scale per tensor.
+//
+// Routing is the same as the bf16 path. Then:
+//   permute  quantises each token's x once (per 16 elements: scale =
+//            e4m3(amax / (6 g_x)), code = e2m1(x / (scale g_x))) and writes
+//            its K copies into expert segments that start on a 128-row
+//            boundary, so that a 128-row token tile is exactly one group of
+//            scale atoms;
+//   gate/up  D = (W13 x) on kind::mxf4nvf4 tensor cores (block scales applied
+//            by the MMA from TMEM), times g_w g_x in the epilogue; h =
+//            silu(g) u in FP32, quantised the same way with g_h (a 16-element
+//            block of h spans 16 TMEM lanes of a warp: shuffles find its
+//            maximum) and written as codes + scales;
+//   down     y = (W2 h) g_w2 g_h in FP32, then the bf16 path's combine.
+//
+// Scale factors of a 128-row x 64-element block are a 512-byte atom (row
+// r0 + 32 r1, block kb at byte 16 r0 + 4 r1 + kb); atoms of a matrix are
+// ordered (row block, 64-element chunk) with the chunk fastest. An atom is
+// copied to 4 TMEM columns with tcgen05.cp and named in the MMA.
+#include <cuda_bf16.h>
+
+#include "grouped_gemm.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+#include "sm100_fp4.cuh"
+
+namespace beam {
+namespace {
+
+constexpr int kBM = 128;          // weight rows per tile (MMA M)
+constexpr int kBN = 128;          // token rows per tile; expert segments align to it
+constexpr int kKB = 256;          // FP4 elements of K per pipeline stage (128 bytes)
+constexpr int kCodeTile = 128 * 128;  // bytes of one 128-row x 256-element code tile
+constexpr int kSfStage = 4 * 512;     // scale atoms of one 128-row x 256-element tile
+constexpr int kThreads = 192;
+
+__device__ __forceinline__ size_t sf_offset(int64_t r, int64_t b, int64_t K) {
+  const int64_t rr = r & 127;
+  return (size_t)(((r >> 7) * (K >> 6) + (b >> 2)) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 +
+                  (b & 3));
+}
+
+// Quantise 16 consecutive values: scale byte and 8 packed code bytes. Every
+// step in FP32 with IEEE division; conversions round to nearest, ties to even,
+// saturating.
+__device__ __forceinline__ uint32_t quantize16(const float (&v)[16], float g, uint2& packed) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t s8 = cvt_e4m3(amax / (6.0f * g));
+  const float d = e4m3_to_f32(s8) * g;
+  uint32_t w[2] = {0u, 0u};
+  if (s8) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i >> 3] |= cvt_e2m1(v[i] / d) << (4 * (i & 7));
+  }
+  packed = make_uint2(w[0], w[1]);
+  return s8;
+}
+
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const float* __restrict__ v,
+                                                            int64_t rows, int64_t K, float g,
+                                                            uint8_t* __restrict__ codes,
+                                                            uint8_t* __restrict__ sf) {
+  const int64_t nb = rows * (K / 16);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nb;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float x[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) x[j] = v[i * 16 + j];
+    uint2 p;
+    sf[i] = (uint8_t)quantize16(x, g, p);
+    *reinterpret_cast<uint2*>(codes + i * 8) = p;
+  }
+}
+
+// One CTA per token: rows of its K assignments (unpadded, for the combine) and
+// padded rows of the quantised copies.
+__global__ void __launch_bounds__(128) permute_nvfp4_kernel(
+    const uint16_t* __restrict__ x, int H, int K, int E, const int32_t* __restrict__ ids,
+    const int32_t* __restrict__ chunk_base, const uint32_t* __restrict__ chunk_mask,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ nb_off,
+    int32_t* __restrict__ pos, uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf, float gx) {
+  __shared__ int s_q[32];
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x;
+  if (tid < K) {
+    const int e = ids[(size_t)t * K + tid];
+    int p = -1, qp = -1;
+    if (e >= 0 && e < E) {
+      const int c = t / kChunk, tl = t - c * kChunk;
+      const uint32_t* m = chunk_mask + ((size_t)c * E + e) * kChunkWords;
+      int rank = 0;
+      for (int wd = 0; wd < (tl >> 5); ++wd) rank += __popc(m[wd]);
+      rank += __popc(m[tl >> 5] & ((1u << (tl & 31)) - 1u));
+      p = chunk_base[(size_t)c * E + e] + rank;
+      qp = p - offsets[e] + nb_off[e] * kBN;
+    }
+    s_q[tid] = qp;
+    pos[(size_t)t * K + tid] = p;
+  }
+  __syncthreads();
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+  for (int b = tid; b < H / 16; b += 128) {
+    const uint4 a = __ldg(src + 2 * b), c = __ldg(src + 2 * b + 1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+    uint2 packed;
+    const uint32_t s8 = quantize16(v, gx, packed);
+    for (int k = 0; k < K; ++k) {
+      const int qp = s_q[k];
+      if (qp < 0) continue;
+      *reinterpret_cast<uint2*>(xq + (size_t)qp * (H / 2) + b * 8) = packed;
+      xsf[sf_offset(qp, b, H)] = (uint8_t)s8;
+    }
+  }
+}
+
+struct Fp4Params {
+  const int32_t* counts;
+  const int32_t* offsets;
+  const int32_t* nb_off;
+  const uint8_t* w_sf;  // weight scales, atom layout over the stacked weight rows
+  const uint8_t* x_sf;  // activation scales, atom layout over the padded rows
+  void* out;            // gate/up: h codes [padded rows][I/2]; down: y fp32 [A][H]
+  uint8_t* out_sf;      // gate/up: h scales, atom layout over the padded rows (K = I)
+  int64_t out_ld;       // gate/up: I / 2 bytes; down: H floats
+  int E;
+  int nk;               // K / 256
+  int Kel;              // K in elements
+  int w_rows;           // weight rows per expert (2I or H)
+  int up_rows;          // up rows' offset inside an expert (I)
+  int n_mblk;           // 128-row weight blocks per expert (I / 128 or H / 128)
+  float acc_scale;      // weight tensor scale x activation tensor scale
+  float h_scale;        // gate/up: tensor scale of the quantised h
+  int I;                // gate/up: intermediate size
+  unsigned* status;
+};
+
+__device__ __forceinline__ void decode_tile4(int tile, const Fp4Params& p, int& e, int& mb,
+                                             int& nb) {
+  int lo = 0, hi = p.E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.nb_off + mid) * p.n_mblk <= tile) lo = mid;
+    else hi = mid - 1;
+  }
+  e = lo;
+  const int base = __ldg(p.nb_off + e);
+  const int nblk = __ldg(p.nb_off + e + 1) - base;
+  const int local = tile - base * p.n_mblk;
+  mb = local / nblk;
+  nb = local - mb * nblk;
+}
+
+template <bool GATEUP>
+struct Cfg4 {
+  static constexpr int kNA = GATEUP ? 2 : 1;
+  static constexpr int kStageBytes = (kNA + 1) * (kCodeTile + kSfStage);
+  static constexpr int kStagesRaw = (220 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr int kAccCols = kNA * kBN;  // FP32 accumulator columns per tile
+  static constexpr int kAccStages = GATEUP ? 1 : 2;
+  static constexpr int kSfCols = 16 * (kNA + 1);  // 4 atoms x 4 columns per operand
+  static constexpr int kTmemCols = 512;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+  static_assert(kAccStages * kAccCols + kSfCols <= kTmemCols, "TMEM overflow");
+  static_assert(kStages >= 2, "pipeline too shallow");
+};
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_w,
+                              const __grid_constant__ CUtensorMap tm_x, const Fp4Params p) {
+  using C = Cfg4<GATEUP>;
+  constexpr int STAGES = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  // stage: [A codes (x kNA)][B codes][A scales (x kNA)][B scales]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_x);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint32_t tsf = tmem_base + (uint32_t)(C::kAccStages * C::kAccCols);
+  const int total = __ldg(p.nb_off + p.E) * p.n_mblk;
+  const int sf_chunks = p.Kel / 64;  // scale atoms per 128-row block
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_normal();
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, mb, nb;
+        decode_tile4(tile, p, e, mb, nb);
+        const int wrow = e * p.w_rows + mb * kBM;
+        const int qrow = (__ldg(p.nb_off + e) + nb) * kBN;
+        const int nblk = __ldg(p.nb_off + e + 1) - __ldg(p.nb_off + e);
+        const uint64_t pol_w = nblk == 1 ? pol_stream : pol_keep;
+        for (int kb = 0; kb < p.nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, kFlagProducer)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::kStageBytes;
+          uint8_t* ssf = sa + (C::kNA + 1) * kCodeTile;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          const int kx = kb * (kKB / 2);  // byte coordinate along K
+          tma_load_2d(sa, &tm_w, &full[stage], kx, wrow, pol_w);
+          bulk_load(ssf, p.w_sf + ((size_t)(wrow / kBM) * sf_chunks + kb * 4) * 512, kSfStage,
+                    &full[stage], pol_w);
+          if (GATEUP) {
+            tma_load_2d(sa + kCodeTile, &tm_w, &full[stage], kx, wrow + p.up_rows, pol_w);
+            bulk_load(ssf + kSfStage,
+                      p.w_sf + ((size_t)((wrow + p.up_rows) / kBM) * sf_chunks + kb * 4) * 512,
+                      kSfStage, &full[stage], pol_w);
+          }
+          tma_load_2d(sa + C::kNA * kCodeTile, &tm_x, &full[stage], kx, qrow, pol_keep);
+          bulk_load(ssf + C::kNA * kSfStage,
+                    p.x_sf + ((size_t)(qrow / kBN) * sf_chunks + kb * 4) * 512, kSfStage,
+                    &full[stage], pol_keep);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      const int64_t first = issued > STAGES ? issued - STAGES : 0;
+      for (int64_t i = first; i < issued; ++i)
+        mbar_wait(&full[i % STAGES], (uint32_t)((i / STAGES) & 1), nullptr, nullptr, 0u,
+                  100000000ull);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------------------------------- MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, mb, nb;
+        decode_tile4(tile, p, e, mb, nb);
+        const int rows = min(kBN, __ldg(p.counts + e) - nb * kBN);
+        const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
+        const uint32_t idesc = idesc_nvf4(kBM, n_mma);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, kFlagMma)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + (uint32_t)(acc * C::kAccCols);
+        const uint32_t d1 = d0 + kBN;
+        for (int kb = 0; kb < p.nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, kFlagMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
+          const uint32_t ssf = sa + (C::kNA + 1) * kCodeTile;
+          // scale atoms of this stage into TMEM: A (gate), A (up), B
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tmem_cp_sf_atom(tsf + 4 * j, smem_desc_sf_atom(ssf + 512 * j));
+            if (GATEUP) tmem_cp_sf_atom(tsf + 16 + 4 * j, smem_desc_sf_atom(ssf + kSfStage + 512 * j));
+            tmem_cp_sf_atom(tsf + 16 * C::kNA + 4 * j,
+                            smem_desc_sf_atom(ssf + C::kNA * kSfStage + 512 * j));
+          }
+          const uint64_t da0 = smem_desc_k_sw128(sa);
+          const uint64_t da1 = smem_desc_k_sw128(sa + kCodeTile);
+          const uint64_t db = smem_desc_k_sw128(sa + C::kNA * kCodeTile);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {  // 64 FP4 elements (32 bytes) per MMA
+            const uint32_t accum = (kb | j) != 0;
+            const uint32_t sfb = tsf + 16 * C::kNA + 4 * j;
+            umma_nvf4(d0, da0 + 2u * j, db + 2u * j, idesc, tsf + 4 * j, sfb, accum);
+            if (GATEUP) umma_nvf4(d1, da1 + 2u * j, db + 2u * j, idesc, tsf + 16 + 4 * j, sfb, accum);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (C::kAccStages == 2) {
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1u;
+        } else {
+          acc_phase ^= 1u;
+        }
+      }
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, nullptr, 0u, 100000000ull);
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;  // weight row inside the 128-row tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int e, mb, nb;
+      decode_tile4(tile, p, e, mb, nb);
+      const int rows = min(kBN, __ldg(p.counts + e) - nb * kBN);
+      const int n_mma = (rows + 15) & ~15;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, kFlagEpilogue)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
+      if (GATEUP) {
+        const int idx = mb * kBM + r;  // intermediate index of this lane
+        const int64_t qrow0 = (int64_t)(__ldg(p.nb_off + e) + nb) * kBN;
+        uint8_t* hq = static_cast<uint8_t*>(p.out);
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          uint32_t g[16], u[16];
+          tmem_ld16(tb + c0, g);
+          tmem_ld16(tb + kBN + c0, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = c0 + j;
+            const float h = gg::silu_mul(__uint_as_float(g[j]) * p.acc_scale,
+                                         __uint_as_float(u[j]) * p.acc_scale);
+            // 16-element block of h: lanes 0-15 or 16-31 of this warp
+            float amax = fabsf(h);
+#pragma unroll
+            for (int off = 1; off < 16; off <<= 1)
+              amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            const uint32_t s8 = cvt_e4m3(amax / (6.0f * p.h_scale));
+            const float d = e4m3_to_f32(s8) * p.h_scale;
+            const uint32_t code = s8 ? cvt_e2m1(h / d) : 0u;
+            const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, 1);
+            if (t < rows) {
+              const int64_t row = qrow0 + t;
+              if ((lane & 1) == 0) hq[row * p.out_ld + idx / 2] = (uint8_t)(code | (partner << 4));
+              if ((lane & 15) == 0) p.out_sf[sf_offset(row, idx / 16, p.I)] = (uint8_t)s8;
+            }
+          }
+        }
+      } else {
+        const int64_t row0 = __ldg(p.offsets + e) + (int64_t)nb * kBN;
+        float* out = static_cast<float*>(p.out) + mb * kBM + r;
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(tb + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < rows) out[(row0 + c0 + j) * p.out_ld] = __uint_as_float(v[j]) * p.acc_scale;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (C::kAccStages == 2) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      } else {
+        acc_phase ^= 1u;
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+template <bool GATEUP>
+cudaError_t run4(const CUtensorMap& tw, const CUtensorMap& tx, const Fp4Params& p,
+                 cudaStream_t st) {
+  using C = Cfg4<GATEUP>;
+  static int configured_device = -1;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (configured_device != dev) {
+    err = cudaFuncSetAttribute(grouped_gemm_nvfp4_kernel<GATEUP>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    configured_device = dev;
+  }
+  grouped_gemm_nvfp4_kernel<GATEUP><<<device_sm_count(), kThreads, C::kSmemBytes, st>>>(tw, tx, p);
+  return cudaGetLastError();
+}
+
+// 2-D byte tensor [rows][cols bytes], box {128 bytes, 128 rows}, 128-byte swizzle.
+cudaError_t encode_codes_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+  return encode_tmap_2d_u8(map, base, cols, rows, 128, 128);
+}
+
+}  // namespace
+
+Fp4Layout make_layout_nvfp4(const beam_moe_cfg& c, int64_t T, int sms) {
+  Fp4Layout F;
+  F.base = make_layout(c, T, sms);
+  Layout& L = F.base;
+  L.bn = kBN;  // token tiles of 128 rows; expert segments padded to them
+  L.pair_gateup = L.pair_down = 0;
+  const int H = c.hidden, I = c.inter, E = c.n_experts;
+  F.rows = ((L.A + kBN - 1) / kBN + E) * (int64_t)kBN;  // bound on the padded rows
+  size_t o = L.route_end;
+  auto take = [&](size_t bytes, size_t align) {
+    o = (o + align - 1) / align * align;
+    size_t at = o;
+    o += bytes;
+    return at;
+  };
+  F.xq = take((size_t)F.rows * H / 2, 1024);
+  F.xsf = take((size_t)F.rows * H / 16, 1024);
+  F.hq = take((size_t)F.rows * I / 2, 1024);
+  F.hsf = take((size_t)F.rows * I / 16, 1024);
+  L.xp = take((size_t)L.A * H * 4, 1024);  // fp32 y, read by the combine
+  L.h = 0;
+  L.total = (o + 255) / 256 * 256;
+  return F;
+}
+
+bool nvfp4_supported(const beam_moe_cfg& c) {
+  return c.hidden % kKB == 0 && c.inter % kKB == 0;
+}
+
+cudaError_t launch_permute_nvfp4(const beam_moe_cfg& c, const Fp4Layout& F, const uint16_t* x,
+                                 float gx, char* ws, cudaStream_t st) {
+  const Layout& L = F.base;
+  permute_nvfp4_kernel<<<(unsigned)L.T, 128, 0, st>>>(
+      x, c.hidden, c.top_k, c.n_experts, reinterpret_cast<const int32_t*>(ws + L.ids),
+      reinterpret_cast<const int32_t*>(ws + L.chunk_cnt),
+      reinterpret_cast<const uint32_t*>(ws + L.chunk_mask),
+      reinterpret_cast<const int32_t*>(ws + L.offsets),
+      reinterpret_cast<const int32_t*>(ws + L.nb_off), reinterpret_cast<int32_t*>(ws + L.pos),
+      reinterpret_cast<uint8_t*>(ws + F.xq), reinterpret_cast<uint8_t*>(ws + F.xsf), gx);
+  return cudaGetLastError();
+}
+
+static Fp4Params base_params4(const beam_moe_cfg& c, const Fp4Layout& F, char* ws) {
+  const Layout& L = F.base;
+  Fp4Params p;
+  p.counts = reinterpret_cast<const int32_t*>(ws + L.counts);
+  p.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
+  p.nb_off = reinterpret_cast<const int32_t*>(ws + L.nb_off);
+  p.E = c.n_experts;
+  p.status = reinterpret_cast<unsigned*>(ws + L.status);
+  p.I = c.inter;
+  return p;
+}
+
+cudaError_t launch_gateup_nvfp4(const beam_moe_cfg& c, const Fp4Layout& F,
+                                const beam_moe_nvfp4_experts& w, char* ws, cudaStream_t st) {
+  const int H = c.hidden, I = c.inter, E = c.n_experts;
+  Fp4Params p = base_params4(c, F, ws);
+  CUtensorMap tw, tx;
+  cudaError_t err = encode_codes_map(&tw, w.w13_codes, (uint64_t)H / 2, (uint64_t)E * 2 * I);
+  if (err != cudaSuccess) return err;
+  err = encode_codes_map(&tx, ws + F.xq, (uint64_t)H / 2, (uint64_t)F.rows);
+  if (err != cudaSuccess) return err;
+  p.w_sf = w.w13_scales;
+  p.x_sf = reinterpret_cast<const uint8_t*>(ws + F.xsf);
+  p.out = ws + F.hq;
+  p.out_sf = reinterpret_cast<uint8_t*>(ws + F.hsf);
+  p.out_ld = I / 2;
+  p.nk = H / kKB;
+  p.Kel = H;
+  p.w_rows = 2 * I;
+  p.up_rows = I;
+  p.n_mblk = I / kBM;
+  p.acc_scale = w.w13_scale * w.x_scale;
+  p.h_scale = w.h_scale;
+  return run4<true>(tw, tx, p, st);
+}
+
+cudaError_t launch_down_nvfp4(const beam_moe_cfg& c, const Fp4Layout& F,
+                              const beam_moe_nvfp4_experts& w, char* ws, cudaStream_t st) {
+  const int H = c.hidden, I = c.inter, E = c.n_experts;
+  Fp4Params p = base_params4(c, F, ws);
+  CUtensorMap tw, tx;
+  cudaError_t err = encode_codes_map(&tw, w.w2_codes, (uint64_t)I / 2, (uint64_t)E * H);
+  if (err != cudaSuccess) return err;
+  err = encode_codes_map(&tx, ws + F.hq, (uint64_t)I / 2, (uint64_t)F.rows);
+  if (err != cudaSuccess) return err;
+  p.w_sf = w.w2_scales;
+  p.x_sf = reinterpret_cast<const uint8_t*>(ws + F.hsf);
+  p.out = ws + F.base.xp;
+  p.out_sf = nullptr;
+  p.out_ld = H;
+  p.nk = I / kKB;
+  p.Kel = I;
+  p.w_rows = H;
+  p.up_rows = 0;
+  p.n_mblk = H / kBM;
+  p.acc_scale = w.w2_scale * w.h_scale;
+  p.h_scale = w.h_scale;
+  return run4<false>(tw, tx, p, st);
+}
+
+cudaError_t launch_quantize_rows(int64_t rows, int64_t K, const float* v, float g, uint8_t* codes,
+                                 uint8_t* sf, cudaStream_t st) {
+  const int64_t nb = rows * (K / 16);
+  const int64_t grid = (nb + 255) / 256 < 148 * 8 ? (nb + 255) / 256 : 148 * 8;
+  quantize_rows_kernel<<<(unsigned)(grid > 0 ? grid : 1), 256, 0, st>>>(v, rows, K, g, codes, sf);
+  return cudaGetLastError();
+}
+
+}  // namespace beam

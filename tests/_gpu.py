@@ -40,6 +40,67 @@ def device_weights(wl):
     return _weights[key]
 
 
+_weights4 = {}
+
+
+def device_weights_nvfp4(wl):
+    """NVFP4 experts on the device (codes, scales in the MMA layout) and the
+    router, cached per block shape."""
+    key = (wl.H, wl.I, wl.E)
+    if key not in _weights4:
+        _weights4.clear()
+        torch.cuda.empty_cache()
+        c13 = torch.empty(wl.E * 2 * wl.I * wl.H // 2, dtype=torch.uint8, device="cuda")
+        s13 = torch.empty(wl.E * 2 * wl.I * wl.H // 16, dtype=torch.uint8, device="cuda")
+        c2 = torch.empty(wl.E * wl.H * wl.I // 2, dtype=torch.uint8, device="cuda")
+        s2 = torch.empty(wl.E * wl.H * wl.I // 16, dtype=torch.uint8, device="cuda")
+        synth.dev_w13_nvfp4(wl, c13.data_ptr(), s13.data_ptr(), stream())
+        synth.dev_w2_nvfp4(wl, c2.data_ptr(), s2.data_ptr(), stream())
+        wr = torch.from_numpy(synth.host_router(wl)).cuda()
+        torch.cuda.synchronize()
+        _weights4[key] = (c13, s13, c2, s2, wr)
+    return _weights4[key]
+
+
+def nvfp4_experts(c13, s13, c2, s2):
+    g_w, g_a = synth.NVFP4_WEIGHT_SCALE, synth.NVFP4_ACT_SCALE
+    return bm.nvfp4_experts(c13, s13, c2, s2, g_w, g_w, g_a, g_a)
+
+
+def forward_nvfp4(wl, x_bits, bias=None):
+    cfg = cfg_of(wl)
+    c13, s13, c2, s2, wr = device_weights_nvfp4(wl)
+    T = x_bits.shape[0]
+    x = to_dev_bits(x_bits)
+    b = None if bias is None else torch.from_numpy(np.asarray(bias, np.float32)).cuda()
+    out = torch.empty((T, wl.H), dtype=torch.int16, device="cuda")
+    ids = torch.empty((T, wl.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, wl.K), dtype=torch.float32, device="cuda")
+    counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+    ws = torch.empty(bm.beam_moe_workspace_size(cfg, T, bm.OP_FORWARD_NVFP4), dtype=torch.uint8,
+                     device="cuda")
+    bm.beam_moe_forward_nvfp4(cfg, x, wr, b, nvfp4_experts(c13, s13, c2, s2), out, ws, ids, w,
+                              counts)
+    flags = bm.beam_moe_check(ws)
+    return {"out": bits_of(out), "ids": ids.cpu().numpy(), "w": w.cpu().numpy(),
+            "counts": counts.cpu().numpy(), "flags": flags}
+
+
+def oracle_outputs_nvfp4(wl, x_bits, tokens, r_oracle, batch=4):
+    cfg = oracle.cfg_for(wl)
+    g_w, g_a = synth.NVFP4_WEIGHT_SCALE, synth.NVFP4_ACT_SCALE
+    rows = []
+    for i in range(0, len(tokens), batch):
+        tt = np.asarray(tokens[i:i + batch])
+        ids = r_oracle["ids"][tt]
+        ex = sorted(set(int(v) for v in ids.ravel()))
+        w13 = {e: synth.host_expert_w13_nvfp4(wl, e) for e in ex}
+        w2 = {e: synth.host_expert_w2_nvfp4(wl, e) for e in ex}
+        rows.append(oracle.experts_nvfp4(cfg, x_bits[tt], ids, r_oracle["weights"][tt], w13, w2,
+                                         g_w, g_w, g_a, g_a))
+    return np.concatenate(rows, axis=0)
+
+
 def to_dev_bits(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
 
