@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
                     [--impl ours|reference] [--no-cpu-baseline]
+                    [--format bf16|nvfp4] [--bias-mode 0|1] [--replay]
 
 A step is one whole block forward (router GEMM, top-k, scan, permute, gate/up
 grouped GEMM, down grouped GEMM, combine) over one batch of T synthetic tokens
@@ -18,6 +19,10 @@ With N GPUs (torchrun, one process per GPU) every rank holds all experts and
 runs its own batch of T tokens: the block is data-parallel over tokens with
 no exchange, so scaling is weak and the only collective is the max of the
 timings.
+
+--format nvfp4 times the same block with NVFP4 experts and activations (4-bit
+E2M1 codes, one E4M3 scale per 16 elements, an fp32 scale per tensor) on the
+block-scaled FP4 tensor cores; its tensor peak is 4x the measured bf16 peak.
 
 --impl reference times the fp64 CPU oracle (the reference arm of this
 repository) on a bounded sample of the same workload on the host cores.
@@ -91,21 +96,24 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def algorithmic(wl, counts):
+def algorithmic(wl, counts, fmt="bf16"):
     """Algorithmic work of one forward with these routed counts.
 
     FLOPs: 6 H I per assignment (tensor cores) + 2 H E per token (FP32 router).
-    Bytes: 3 H I x 2 per touched expert, router weights, x and out.
-    gate/up kernel bytes: 2 I H x 2 per touched expert + permuted rows in + h out.
+    Bytes: 3 H I x b per touched expert (b = 2 for bf16; 0.5625 for NVFP4: a
+    4-bit code plus one E4M3 scale per 16 elements), router weights, x and out.
+    gate/up kernel bytes: 2 I H x b per touched expert + its input rows + its
+    output rows (bf16 rows, or NVFP4 rows at 0.5625 bytes per element).
     """
     touched = int(np.count_nonzero(counts))
     A = wl.T * wl.K
+    b = 2.0 if fmt == "bf16" else 0.5625
     return {
         "touched_experts": touched,
         "expert_flops": 6.0 * wl.H * wl.I * A,
         "router_flops": 2.0 * wl.H * wl.E * wl.T,
-        "block_bytes": touched * 3.0 * wl.H * wl.I * 2 + wl.E * wl.H * 4 + 2 * wl.T * wl.H * 2,
-        "gateup_bytes": touched * 2.0 * wl.I * wl.H * 2 + A * wl.H * 2 + A * wl.I * 2,
+        "block_bytes": touched * 3.0 * wl.H * wl.I * b + wl.E * wl.H * 4 + 2 * wl.T * wl.H * 2,
+        "gateup_bytes": touched * 2.0 * wl.I * wl.H * b + A * wl.H * b + A * wl.I * b,
         "gateup_flops": 4.0 * wl.H * wl.I * A,
     }
 
@@ -267,10 +275,23 @@ def run_ours(args, wl):
     cfg = bm.beam_cfg(wl.H, wl.I, wl.E, wl.G, wl.Gk, wl.K, wl.renormalize, args.bias_mode,
                       wl.scale)
     # all ranks hold the same experts (seed 0); each rank routes its own tokens
-    w13 = torch.empty(wl.w13_elems, dtype=torch.int16, device=dev)
-    w2 = torch.empty(wl.w2_elems, dtype=torch.int16, device=dev)
-    synth.dev_w13(wl, w13.data_ptr(), st)
-    synth.dev_w2(wl, w2.data_ptr(), st)
+    nvfp4 = args.format == "nvfp4"
+    if nvfp4:
+        c13 = torch.empty(wl.w13_elems // 2, dtype=torch.uint8, device=dev)
+        s13 = torch.empty(wl.w13_elems // 16, dtype=torch.uint8, device=dev)
+        c2 = torch.empty(wl.w2_elems // 2, dtype=torch.uint8, device=dev)
+        s2 = torch.empty(wl.w2_elems // 16, dtype=torch.uint8, device=dev)
+        synth.dev_w13_nvfp4(wl, c13.data_ptr(), s13.data_ptr(), st)
+        synth.dev_w2_nvfp4(wl, c2.data_ptr(), s2.data_ptr(), st)
+        experts = bm.nvfp4_experts(c13, s13, c2, s2, synth.NVFP4_WEIGHT_SCALE,
+                                   synth.NVFP4_WEIGHT_SCALE, synth.NVFP4_ACT_SCALE,
+                                   synth.NVFP4_ACT_SCALE)
+        w13 = w2 = None
+    else:
+        w13 = torch.empty(wl.w13_elems, dtype=torch.int16, device=dev)
+        w2 = torch.empty(wl.w2_elems, dtype=torch.int16, device=dev)
+        synth.dev_w13(wl, w13.data_ptr(), st)
+        synth.dev_w2(wl, w2.data_ptr(), st)
     wr = torch.from_numpy(synth.host_router(wl)).to(dev)
     bias = synth.host_bias(wl)
     b = None if bias is None else torch.from_numpy(bias).to(dev)
@@ -278,7 +299,9 @@ def run_ours(args, wl):
     synth.dev_x(wl, x.data_ptr(), st, seed=rank_seed(rank))
     out = torch.empty((wl.T, wl.H), dtype=torch.int16, device=dev)
     counts = torch.zeros(wl.E, dtype=torch.int32, device=dev)
-    ws = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T), dtype=torch.uint8, device=dev)
+    ws = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T,
+                                                bm.OP_FORWARD_NVFP4 if nvfp4 else bm.OP_FORWARD),
+                     dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
 
@@ -288,7 +311,10 @@ def run_ours(args, wl):
         bm.beam_moe_forward(cfg, x, wr, b, w13, w2, out, ws, ids, wts, counts, stream=st)
 
     def step(trace=None):
-        if args.replay:
+        if nvfp4:
+            bm.beam_moe_forward_nvfp4(cfg, x, wr, b, experts, out, ws, expert_counts=counts,
+                                      stream=st, trace=trace)
+        elif args.replay:
             bm.beam_moe_forward_routed(cfg, x, ids, wts, w13, w2, out, ws, counts, stream=st)
         elif trace is None:
             bm.beam_moe_forward(cfg, x, wr, b, w13, w2, out, ws, expert_counts=counts,
@@ -353,8 +379,12 @@ def run_ours(args, wl):
     value = tokens / (ms_step / 1000.0)
     e2e_value = tokens / (e2e_ms / args.steps / 1000.0)
 
-    alg = algorithmic(wl, counts.cpu().numpy())
+    alg = algorithmic(wl, counts.cpu().numpy(), args.format)
     peaks, peak_kind = load_peaks()
+    if nvfp4:  # dense FP4 = 4x dense BF16 (nominal 9 vs 2.25 PFLOP/s), scaled from the measured
+        peaks = dict(peaks, bf16_tflops=4 * peaks["bf16_tflops"],
+                     bf16_tflops_sustained=4 * peaks.get("bf16_tflops_sustained",
+                                                         peaks["bf16_tflops"]))
     # Tensor peak: the burst figure for short steps, the sustained (power-capped)
     # figure once a step lasts 10 ms or more and the GPU runs at its power cap.
     sustained = ms_step >= 10.0 and "bf16_tflops_sustained" in peaks
@@ -375,17 +405,22 @@ def run_ours(args, wl):
     if args.replay:  # no per-stage events on this entry point
         roof.update(achieved=None, frac=None)
     roof["frac"] = None if roof["achieved"] is None else roof["achieved"] / roof["peak"]
-    roof["traffic"] = gateup_traffic(wl, alg["touched_experts"])
+    # the recorded DRAM traffic belongs to the bf16 gate/up kernel only
+    roof["traffic"] = None if nvfp4 else gateup_traffic(wl, alg["touched_experts"])
     roof["algorithmic_bytes"] = alg["gateup_bytes"]
-    roof["kernel"] = "gateup_grouped_gemm"
+    roof["kernel"] = "gateup_grouped_gemm_nvfp4" if nvfp4 else "gateup_grouped_gemm"
+    if nvfp4:
+        roof["peak_note"] = "dense FP4 tensor peak = 4 x measured bf16 (nominal ratio)"
     roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
         else "fallback"
     block_s = ms_step / 1000.0
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4" if nvfp4 else "bf16",
+        "data": "synthetic",
         "config": {"workload": describe(wl) + (" [routes replayed]" if args.replay else "")
+                   + (" [NVFP4 experts and activations]" if nvfp4 else "")
                    + (" [selection-only bias]" if args.bias_mode == 1 else ""),
                    "T": wl.T, "tokens_per_rank": wl.T,
                    "l2": "flushed before every timed step (256 MB write, outside the events)",
@@ -429,6 +464,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--bias-mode", type=int, default=0, choices=[0, 1],
                     help="0: router bias on the logits; 1: on the choice scores only")
+    ap.add_argument("--format", default="bf16", choices=["bf16", "nvfp4"],
+                    help="expert weight / activation format of the timed forward")
     ap.add_argument("--replay", action="store_true",
                     help="time the expert path with recorded routes (beam_moe_forward_routed)")
     ap.add_argument("--tokens", type=int, default=None,
@@ -438,6 +475,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
+    if args.replay and args.format != "bf16":
+        raise SystemExit("--replay times the bf16 routed entry point only")
     wl = synth.workload(args.workload)
     if args.tokens is not None:
         wl = wl.with_T(args.tokens)

@@ -36,7 +36,6 @@ constexpr int kBN = 128;          // token rows per tile; expert segments align 
 constexpr int kKB = 256;          // FP4 elements of K per pipeline stage (128 bytes)
 constexpr int kCodeTile = 128 * 128;  // bytes of one 128-row x 256-element code tile
 constexpr int kSfStage = 4 * 512;     // scale atoms of one 128-row x 256-element tile
-constexpr int kThreads = 192;
 
 __device__ __forceinline__ size_t sf_offset(int64_t r, int64_t b, int64_t K) {
   const int64_t rr = r & 127;
@@ -164,6 +163,11 @@ __device__ __forceinline__ void decode_tile4(int tile, const Fp4Params& p, int& 
 
 template <bool GATEUP>
 struct Cfg4 {
+  // warp 0 TMA producer, warp 1 MMA issuer, then the epilogue warps: the
+  // gate/up epilogue (SwiGLU + NVFP4 quantisation of h) is the heavy one and
+  // gets two warps per TMEM lane quarter, each on half of the token columns
+  static constexpr int kEpiWarps = GATEUP ? 8 : 4;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kNA = GATEUP ? 2 : 1;
   static constexpr int kStageBytes = (kNA + 1) * (kCodeTile + kSfStage);
   static constexpr int kStagesRaw = (220 * 1024) / kStageBytes;
@@ -171,14 +175,18 @@ struct Cfg4 {
   static constexpr int kAccCols = kNA * kBN;  // FP32 accumulator columns per tile
   static constexpr int kAccStages = GATEUP ? 1 : 2;
   static constexpr int kSfCols = 16 * (kNA + 1);  // 4 atoms x 4 columns per operand
+  // Scale columns rotate over several buffers: the copy for a stage then never
+  // overwrites columns that MMAs of the previous stages may still read, so the
+  // tensor pipe does not drain between stages.
+  static constexpr int kSfBufs = 4;
   static constexpr int kTmemCols = 512;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
-  static_assert(kAccStages * kAccCols + kSfCols <= kTmemCols, "TMEM overflow");
+  static_assert(kAccStages * kAccCols + kSfBufs * kSfCols <= kTmemCols, "TMEM overflow");
   static_assert(kStages >= 2, "pipeline too shallow");
 };
 
 template <bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
     grouped_gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_w,
                               const __grid_constant__ CUtensorMap tm_x, const Fp4Params p) {
   using C = Cfg4<GATEUP>;
@@ -203,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 32 * C::kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -281,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
+      int sfbuf = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int e, mb, nb;
@@ -300,12 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
           const uint32_t ssf = sa + (C::kNA + 1) * kCodeTile;
+          const uint32_t tsf_s = tsf + (uint32_t)(sfbuf * C::kSfCols);
+          if (++sfbuf == C::kSfBufs) sfbuf = 0;
           // scale atoms of this stage into TMEM: A (gate), A (up), B
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            tmem_cp_sf_atom(tsf + 4 * j, smem_desc_sf_atom(ssf + 512 * j));
-            if (GATEUP) tmem_cp_sf_atom(tsf + 16 + 4 * j, smem_desc_sf_atom(ssf + kSfStage + 512 * j));
-            tmem_cp_sf_atom(tsf + 16 * C::kNA + 4 * j,
+            tmem_cp_sf_atom(tsf_s + 4 * j, smem_desc_sf_atom(ssf + 512 * j));
+            if (GATEUP) tmem_cp_sf_atom(tsf_s + 16 + 4 * j, smem_desc_sf_atom(ssf + kSfStage + 512 * j));
+            tmem_cp_sf_atom(tsf_s + 16 * C::kNA + 4 * j,
                             smem_desc_sf_atom(ssf + C::kNA * kSfStage + 512 * j));
           }
           const uint64_t da0 = smem_desc_k_sw128(sa);
@@ -314,9 +325,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {  // 64 FP4 elements (32 bytes) per MMA
             const uint32_t accum = (kb | j) != 0;
-            const uint32_t sfb = tsf + 16 * C::kNA + 4 * j;
-            umma_nvf4(d0, da0 + 2u * j, db + 2u * j, idesc, tsf + 4 * j, sfb, accum);
-            if (GATEUP) umma_nvf4(d1, da1 + 2u * j, db + 2u * j, idesc, tsf + 16 + 4 * j, sfb, accum);
+            const uint32_t sfb = tsf_s + 16 * C::kNA + 4 * j;
+            umma_nvf4(d0, da0 + 2u * j, db + 2u * j, idesc, tsf_s + 4 * j, sfb, accum);
+            if (GATEUP) umma_nvf4(d1, da1 + 2u * j, db + 2u * j, idesc, tsf_s + 16 + 4 * j, sfb, accum);
           }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -352,32 +363,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
       if (GATEUP) {
+        // This warp owns token columns [c_beg, c_beg + 64) of its 32 rows. It
+        // forms h = silu(g) u for them, hands the accumulator back to the MMA
+        // warp, and quantises and stores while the next tile accumulates.
+        const int c_beg = ((warp - 2) >> 2) * 64;
+        float h[64];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c_beg + 16 * c < n_mma) {  // warp-uniform
+            uint32_t g[16], u[16];
+            tmem_ld16(tb + c_beg + 16 * c, g);
+            tmem_ld16(tb + kBN + c_beg + 16 * c, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              h[16 * c + j] = gg::silu_mul(__uint_as_float(g[j]) * p.acc_scale,
+                                           __uint_as_float(u[j]) * p.acc_scale);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+
         const int idx = mb * kBM + r;  // intermediate index of this lane
-        const int64_t qrow0 = (int64_t)(__ldg(p.nb_off + e) + nb) * kBN;
-        uint8_t* hq = static_cast<uint8_t*>(p.out);
-        for (int c0 = 0; c0 < n_mma; c0 += 16) {
-          uint32_t g[16], u[16];
-          tmem_ld16(tb + c0, g);
-          tmem_ld16(tb + kBN + c0, u);
-          tmem_ld_wait();
+        const int64_t qrow0 = (int64_t)(__ldg(p.nb_off + e) + nb) * kBN;  // 128-row aligned
+        uint8_t* hq = static_cast<uint8_t*>(p.out) + qrow0 * p.out_ld + idx / 2;
+        // scale byte of (row qrow0 + t, block idx / 16) in the atom layout
+        uint8_t* hsf = p.out_sf +
+                       ((qrow0 >> 7) * (p.I >> 6) + (idx >> 6)) * 512 + ((idx >> 4) & 3);
+        const float six_g = 6.0f * p.h_scale;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int t = c0 + j;
-            const float h = gg::silu_mul(__uint_as_float(g[j]) * p.acc_scale,
-                                         __uint_as_float(u[j]) * p.acc_scale);
-            // 16-element block of h: lanes 0-15 or 16-31 of this warp
-            float amax = fabsf(h);
+        for (int c = 0; c < 4; ++c) {
+          if (c_beg + 16 * c < n_mma) {
 #pragma unroll
-            for (int off = 1; off < 16; off <<= 1)
-              amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-            const uint32_t s8 = cvt_e4m3(amax / (6.0f * p.h_scale));
-            const float d = e4m3_to_f32(s8) * p.h_scale;
-            const uint32_t code = s8 ? cvt_e2m1(h / d) : 0u;
-            const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, 1);
-            if (t < rows) {
-              const int64_t row = qrow0 + t;
-              if ((lane & 1) == 0) hq[row * p.out_ld + idx / 2] = (uint8_t)(code | (partner << 4));
-              if ((lane & 15) == 0) p.out_sf[sf_offset(row, idx / 16, p.I)] = (uint8_t)s8;
+            for (int j = 0; j < 16; ++j) {
+              const int t = c_beg + 16 * c + j;
+              const float v = h[16 * c + j];
+              // 16-element block of h: lanes 0-15 or 16-31 of this warp. The
+              // magnitudes' bit patterns order like the values.
+              uint32_t am = __float_as_uint(v) & 0x7FFFFFFFu;
+#pragma unroll
+              for (int off = 1; off < 16; off <<= 1)
+                am = max(am, __shfl_xor_sync(0xffffffffu, am, off));
+              const uint32_t s8 = cvt_e4m3(__fdividef(__uint_as_float(am), six_g));
+              const float d = e4m3_to_f32(s8) * p.h_scale;
+              uint32_t code = cvt_e2m1(__fdividef(v, d));
+              code = s8 ? code : 0u;
+              const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, 1);
+              if (t < rows) {
+                if ((lane & 1) == 0) hq[t * p.out_ld] = (uint8_t)(code | (partner << 4));
+                if ((lane & 15) == 0) hsf[(t & 31) * 16 + (t >> 5) * 4] = (uint8_t)s8;
+              }
             }
           }
         }
@@ -393,8 +428,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c0 + j < rows) out[(row0 + c0 + j) * p.out_ld] = __uint_as_float(v[j]) * p.acc_scale;
         }
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      if (!GATEUP) {
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+      }
       if (C::kAccStages == 2) {
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
@@ -426,7 +463,7 @@ cudaError_t run4(const CUtensorMap& tw, const CUtensorMap& tx, const Fp4Params& 
     if (err != cudaSuccess) return err;
     configured_device = dev;
   }
-  grouped_gemm_nvfp4_kernel<GATEUP><<<device_sm_count(), kThreads, C::kSmemBytes, st>>>(tw, tx, p);
+  grouped_gemm_nvfp4_kernel<GATEUP><<<device_sm_count(), C::kThreads, C::kSmemBytes, st>>>(tw, tx, p);
   return cudaGetLastError();
 }
 
