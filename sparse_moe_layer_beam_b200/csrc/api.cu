@@ -74,6 +74,7 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms) {
   L.counts = take(sizeof(int32_t) * E, 256);
   L.offsets = take(sizeof(int32_t) * (E + 1), 256);
   L.nb_off = take(sizeof(int32_t) * (E + 1), 256);
+  L.nb2_off = take(sizeof(int32_t) * (E + 1), 256);
   L.ids = take(sizeof(int32_t) * (size_t)L.A, 256);
   L.w = take(sizeof(float) * (size_t)L.A, 256);
   L.pos = take(sizeof(int32_t) * (size_t)L.A, 256);

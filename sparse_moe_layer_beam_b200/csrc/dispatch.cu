@@ -62,11 +62,12 @@ __global__ void __launch_bounds__(1024) scan_kernel(const uint32_t* __restrict__
                                                     int E, int bn, int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ nb_off,
+                                                    int32_t* __restrict__ nb2_off,
                                                     int32_t* __restrict__ counts_out) {
   __shared__ int32_t part[1024];   // per (team member, expert) partial counts
   __shared__ int32_t s_off[512];   // first row of each expert
   __shared__ int32_t warp_tot[32];
-  __shared__ int32_t total[2];
+  __shared__ int32_t total[3];
   const int tid = threadIdx.x;
   const int tpe = 1024 / E;  // threads per expert (E <= 512)
   const int e = tid % E, j = tid / E;
@@ -83,16 +84,20 @@ __global__ void __launch_bounds__(1024) scan_kernel(const uint32_t* __restrict__
     for (int q = 0; q < tpe; ++q) tot += part[q * E + tid];
   const int off = block_exclusive_scan(tid < E ? tot : 0, warp_tot, &total[0]);
   const int nbo = block_exclusive_scan(tid < E ? (tot + bn - 1) / bn : 0, warp_tot, &total[1]);
+  const int nb2o =
+      block_exclusive_scan(tid < E ? (tot + 2 * bn - 1) / (2 * bn) : 0, warp_tot, &total[2]);
   if (tid < E) {
     s_off[tid] = off;
     offsets[tid] = off;
     nb_off[tid] = nbo;
+    nb2_off[tid] = nb2o;
     counts[tid] = tot;
     if (counts_out) counts_out[tid] = tot;
   }
   if (tid == 0) {
     offsets[E] = total[0];
     nb_off[E] = total[1];
+    nb2_off[E] = total[2];
   }
   __syncthreads();
   if (act) {
@@ -186,7 +191,8 @@ cudaError_t launch_scan(const beam_moe_cfg& c, const Layout& L, char* ws, int32_
                                   reinterpret_cast<int32_t*>(ws + L.chunk_cnt), L.nchunks,
                                   c.n_experts, L.bn, reinterpret_cast<int32_t*>(ws + L.counts),
                                   reinterpret_cast<int32_t*>(ws + L.offsets),
-                                  reinterpret_cast<int32_t*>(ws + L.nb_off), counts_out);
+                                  reinterpret_cast<int32_t*>(ws + L.nb_off),
+                                  reinterpret_cast<int32_t*>(ws + L.nb2_off), counts_out);
   return cudaGetLastError();
 }
 

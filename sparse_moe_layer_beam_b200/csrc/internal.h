@@ -38,6 +38,7 @@ struct Layout {
   size_t counts;    // int32[E]
   size_t offsets;   // int32[E + 1] first row of each expert in the permuted rows
   size_t nb_off;    // int32[E + 1] prefix of ceil(count / bn)
+  size_t nb2_off;   // int32[E + 1] prefix of ceil(count / (2 bn))
   size_t ids;       // int32[T * K]
   size_t w;         // float[T * K]
   size_t pos;       // int32[T * K] permuted row of each assignment

@@ -127,7 +127,8 @@ __global__ void __launch_bounds__(128) permute_nvfp4_kernel(
 struct Fp4Params {
   const int32_t* counts;
   const int32_t* offsets;
-  const int32_t* nb_off;
+  const int32_t* nb_off;   // prefix of 128-row token blocks per expert
+  const int32_t* tile_off; // prefix of token tiles per expert (of the kernel's tile height)
   const uint8_t* w_sf;  // weight scales, atom layout over the stacked weight rows
   const uint8_t* x_sf;  // activation scales, atom layout over the padded rows
   void* out;            // gate/up: h codes [padded rows][I/2]; down: y fp32 [A][H]
@@ -145,44 +146,54 @@ struct Fp4Params {
   unsigned* status;
 };
 
+// Tile -> (expert, 128-row weight block, token tile of the expert); token tiles
+// are fastest, so CTAs running at the same time share weight blocks in L2.
 __device__ __forceinline__ void decode_tile4(int tile, const Fp4Params& p, int& e, int& mb,
-                                             int& nb) {
+                                             int& tt, int& ntt) {
   int lo = 0, hi = p.E - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(p.nb_off + mid) * p.n_mblk <= tile) lo = mid;
+    if (__ldg(p.tile_off + mid) * p.n_mblk <= tile) lo = mid;
     else hi = mid - 1;
   }
   e = lo;
-  const int base = __ldg(p.nb_off + e);
-  const int nblk = __ldg(p.nb_off + e + 1) - base;
+  const int base = __ldg(p.tile_off + e);
+  ntt = __ldg(p.tile_off + e + 1) - base;
   const int local = tile - base * p.n_mblk;
-  mb = local / nblk;
-  nb = local - mb * nblk;
+  mb = local / ntt;
+  tt = local - mb * ntt;
 }
 
 template <bool GATEUP>
 struct Cfg4 {
-  // warp 0 TMA producer, warp 1 MMA issuer, then the epilogue warps: the
-  // gate/up epilogue (SwiGLU + NVFP4 quantisation of h) is the heavy one and
-  // gets two warps per TMEM lane quarter, each on half of the token columns
+  // warp 0 TMA producer, warp 1 MMA issuer, then the epilogue warps. The
+  // gate/up epilogue (SwiGLU + NVFP4 quantisation of h) is the heavy one: two
+  // warps per TMEM lane quarter, each on half of the token columns, and its
+  // single accumulator is handed back as soon as it is read. The down
+  // epilogue only scales and stores y; it has one warp per lane quarter and a
+  // second accumulator stage instead.
   static constexpr int kEpiWarps = GATEUP ? 8 : 4;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
-  static constexpr int kNA = GATEUP ? 2 : 1;
-  static constexpr int kStageBytes = (kNA + 1) * (kCodeTile + kSfStage);
+  static constexpr int kNA = GATEUP ? 2 : 1;   // 128-row A tiles (gate and up, or down)
+  static constexpr int kTok = 128;             // token rows per tile (MMA N)
+  static constexpr int kTB = kTok / 128;       // 128-row token blocks per tile
+  static constexpr int kStageBytes = (kNA + kTB) * (kCodeTile + kSfStage);
   static constexpr int kStagesRaw = (220 * 1024) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr int kAccCols = kNA * kBN;  // FP32 accumulator columns per tile
+  static constexpr int kAccCols = kNA * kTok;  // FP32 accumulator columns per tile
   static constexpr int kAccStages = GATEUP ? 1 : 2;
-  static constexpr int kSfCols = 16 * (kNA + 1);  // 4 atoms x 4 columns per operand
-  // Scale columns rotate over several buffers: the copy for a stage then never
-  // overwrites columns that MMAs of the previous stages may still read, so the
-  // tensor pipe does not drain between stages.
+  // Scale columns per stage: 4 per 64-element chunk and 128-row block. They
+  // rotate over several buffers, so the copy for a stage never overwrites
+  // columns that MMAs of the previous stages may still read.
+  static constexpr int kSfColsA = 16 * kNA;
+  static constexpr int kSfCols = kSfColsA + 16 * kTB;
   static constexpr int kSfBufs = 4;
   static constexpr int kTmemCols = 512;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+  static constexpr int kColsPerWarp = kTok * 4 / kEpiWarps;  // token columns per epilogue warp
   static_assert(kAccStages * kAccCols + kSfBufs * kSfCols <= kTmemCols, "TMEM overflow");
   static_assert(kStages >= 2, "pipeline too shallow");
+  static_assert(kColsPerWarp <= 128, "epilogue registers");
 };
 
 template <bool GATEUP>
@@ -191,10 +202,11 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
                               const __grid_constant__ CUtensorMap tm_x, const Fp4Params p) {
   using C = Cfg4<GATEUP>;
   constexpr int STAGES = C::kStages;
+  constexpr int TOK = C::kTok;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  // stage: [A codes (x kNA)][B codes][A scales (x kNA)][B scales]
+  // stage: [A codes (x kNA)][B codes (x kTB)][A scales (x kNA)][B scales (x kTB)]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
@@ -228,7 +240,7 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const uint32_t tsf = tmem_base + (uint32_t)(C::kAccStages * C::kAccCols);
-  const int total = __ldg(p.nb_off + p.E) * p.n_mblk;
+  const int total = __ldg(p.tile_off + p.E) * p.n_mblk;
   const int sf_chunks = p.Kel / 64;  // scale atoms per 128-row block
 
   if (warp == 0) {
@@ -241,20 +253,22 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
       int64_t issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        int e, mb, nb;
-        decode_tile4(tile, p, e, mb, nb);
+        int e, mb, tt, ntt;
+        decode_tile4(tile, p, e, mb, tt, ntt);
         const int wrow = e * p.w_rows + mb * kBM;
-        const int qrow = (__ldg(p.nb_off + e) + nb) * kBN;
-        const int nblk = __ldg(p.nb_off + e + 1) - __ldg(p.nb_off + e);
-        const uint64_t pol_w = nblk == 1 ? pol_stream : pol_keep;
+        const int qblk = __ldg(p.nb_off + e) + tt * C::kTB;  // first 128-row token block
+        const int rows = min(TOK, __ldg(p.counts + e) - tt * TOK);
+        const int nbb = (rows + 127) >> 7;                   // token blocks present
+        const uint64_t pol_w = ntt == 1 ? pol_stream : pol_keep;
+        const uint32_t bytes = (uint32_t)((C::kNA + nbb) * (kCodeTile + kSfStage));
         for (int kb = 0; kb < p.nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, kFlagProducer)) {
             ok = false;
             break;
           }
           uint8_t* sa = smem + stage * C::kStageBytes;
-          uint8_t* ssf = sa + (C::kNA + 1) * kCodeTile;
-          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          uint8_t* ssf = sa + (C::kNA + C::kTB) * kCodeTile;
+          mbar_arrive_expect_tx(&full[stage], bytes);
           const int kx = kb * (kKB / 2);  // byte coordinate along K
           tma_load_2d(sa, &tm_w, &full[stage], kx, wrow, pol_w);
           bulk_load(ssf, p.w_sf + ((size_t)(wrow / kBM) * sf_chunks + kb * 4) * 512, kSfStage,
@@ -265,10 +279,13 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
                       p.w_sf + ((size_t)((wrow + p.up_rows) / kBM) * sf_chunks + kb * 4) * 512,
                       kSfStage, &full[stage], pol_w);
           }
-          tma_load_2d(sa + C::kNA * kCodeTile, &tm_x, &full[stage], kx, qrow, pol_keep);
-          bulk_load(ssf + C::kNA * kSfStage,
-                    p.x_sf + ((size_t)(qrow / kBN) * sf_chunks + kb * 4) * 512, kSfStage,
-                    &full[stage], pol_keep);
+          for (int b = 0; b < nbb; ++b) {
+            tma_load_2d(sa + (C::kNA + b) * kCodeTile, &tm_x, &full[stage], kx,
+                        (qblk + b) * 128, pol_keep);
+            bulk_load(ssf + (C::kNA + b) * kSfStage,
+                      p.x_sf + ((size_t)(qblk + b) * sf_chunks + kb * 4) * 512, kSfStage,
+                      &full[stage], pol_keep);
+          }
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -292,15 +309,15 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
       int sfbuf = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        int e, mb, nb;
-        decode_tile4(tile, p, e, mb, nb);
-        const int rows = min(kBN, __ldg(p.counts + e) - nb * kBN);
+        int e, mb, tt, ntt;
+        decode_tile4(tile, p, e, mb, tt, ntt);
+        const int rows = min(TOK, __ldg(p.counts + e) - tt * TOK);
         const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
         const uint32_t idesc = idesc_nvf4(kBM, n_mma);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, kFlagMma)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + (uint32_t)(acc * C::kAccCols);
-        const uint32_t d1 = d0 + kBN;
+        const uint32_t d1 = d0 + TOK;
         for (int kb = 0; kb < p.nk; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.status, kFlagMma)) {
             ok = false;
@@ -308,16 +325,22 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
-          const uint32_t ssf = sa + (C::kNA + 1) * kCodeTile;
+          const uint32_t ssf = sa + (C::kNA + C::kTB) * kCodeTile;
           const uint32_t tsf_s = tsf + (uint32_t)(sfbuf * C::kSfCols);
+          const uint32_t tsfb = tsf_s + C::kSfColsA;
           if (++sfbuf == C::kSfBufs) sfbuf = 0;
-          // scale atoms of this stage into TMEM: A (gate), A (up), B
+          // Scale atoms of this stage into TMEM. Chunk j of the A tile(s) at
+          // columns 4j (gate or down) and 16 + 4j (up); chunk j of token block
+          // b at 4 (kTB j + b), so that a 256-row B operand finds rows
+          // 128-255 in the four columns after rows 0-127.
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             tmem_cp_sf_atom(tsf_s + 4 * j, smem_desc_sf_atom(ssf + 512 * j));
             if (GATEUP) tmem_cp_sf_atom(tsf_s + 16 + 4 * j, smem_desc_sf_atom(ssf + kSfStage + 512 * j));
-            tmem_cp_sf_atom(tsf_s + 16 * C::kNA + 4 * j,
-                            smem_desc_sf_atom(ssf + C::kNA * kSfStage + 512 * j));
+#pragma unroll
+            for (int b = 0; b < C::kTB; ++b)  // an absent second block copies stale bytes
+              tmem_cp_sf_atom(tsfb + 4 * (C::kTB * j + b),
+                              smem_desc_sf_atom(ssf + (C::kNA + b) * kSfStage + 512 * j));
           }
           const uint64_t da0 = smem_desc_k_sw128(sa);
           const uint64_t da1 = smem_desc_k_sw128(sa + kCodeTile);
@@ -325,7 +348,7 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {  // 64 FP4 elements (32 bytes) per MMA
             const uint32_t accum = (kb | j) != 0;
-            const uint32_t sfb = tsf_s + 16 * C::kNA + 4 * j;
+            const uint32_t sfb = tsfb + 4 * C::kTB * j;
             umma_nvf4(d0, da0 + 2u * j, db + 2u * j, idesc, tsf_s + 4 * j, sfb, accum);
             if (GATEUP) umma_nvf4(d1, da1 + 2u * j, db + 2u * j, idesc, tsf_s + 16 + 4 * j, sfb, accum);
           }
@@ -337,10 +360,8 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
         }
         if (!ok) break;
         umma_commit(&tfull[acc]);
-        if (C::kAccStages == 2) {
-          acc ^= 1;
-          if (acc == 0) acc_phase ^= 1u;
-        } else {
+        if (++acc == C::kAccStages) {
+          acc = 0;
           acc_phase ^= 1u;
         }
       }
@@ -350,63 +371,69 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
     __syncwarp();
   } else {
     // -------------------------------------------------------------- epilogue
+    // Each warp owns TMEM lane quarter q (32 weight rows) and token columns
+    // [c_beg, c_beg + HALF) of every tile.
+    constexpr int HALF = C::kColsPerWarp;
     const int q = warp & 3;
     const int r = q * 32 + lane;  // weight row inside the 128-row tile
+    const int c_beg = ((warp - 2) >> 2) * HALF;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      int e, mb, nb;
-      decode_tile4(tile, p, e, mb, nb);
-      const int rows = min(kBN, __ldg(p.counts + e) - nb * kBN);
+      int e, mb, tt, ntt;
+      decode_tile4(tile, p, e, mb, tt, ntt);
+      const int rows = min(TOK, __ldg(p.counts + e) - tt * TOK);
       const int n_mma = (rows + 15) & ~15;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, kFlagEpilogue)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
+      uint64_t* const released = &tempty[acc];
+      if (++acc == C::kAccStages) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
       if (GATEUP) {
-        // This warp owns token columns [c_beg, c_beg + 64) of its 32 rows. It
-        // forms h = silu(g) u for them, hands the accumulator back to the MMA
-        // warp, and quantises and stores while the next tile accumulates.
-        const int c_beg = ((warp - 2) >> 2) * 64;
-        float h[64];
+        // h = silu(g) u into registers, then TMEM goes back to the MMA warp
+        float v[HALF];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < HALF / 16; ++c) {
           if (c_beg + 16 * c < n_mma) {  // warp-uniform
             uint32_t g[16], u[16];
             tmem_ld16(tb + c_beg + 16 * c, g);
-            tmem_ld16(tb + kBN + c_beg + 16 * c, u);
+            tmem_ld16(tb + TOK + c_beg + 16 * c, u);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              h[16 * c + j] = gg::silu_mul(__uint_as_float(g[j]) * p.acc_scale,
+              v[16 * c + j] = gg::silu_mul(__uint_as_float(g[j]) * p.acc_scale,
                                            __uint_as_float(u[j]) * p.acc_scale);
           }
         }
         tc_fence_before();
-        mbar_arrive(&tempty[acc]);
+        mbar_arrive(released);
 
         const int idx = mb * kBM + r;  // intermediate index of this lane
-        const int64_t qrow0 = (int64_t)(__ldg(p.nb_off + e) + nb) * kBN;  // 128-row aligned
+        const int64_t qrow0 = (int64_t)(__ldg(p.nb_off + e) + tt) * kBN;  // 128-row aligned
         uint8_t* hq = static_cast<uint8_t*>(p.out) + qrow0 * p.out_ld + idx / 2;
         // scale byte of (row qrow0 + t, block idx / 16) in the atom layout
         uint8_t* hsf = p.out_sf +
                        ((qrow0 >> 7) * (p.I >> 6) + (idx >> 6)) * 512 + ((idx >> 4) & 3);
         const float six_g = 6.0f * p.h_scale;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < HALF / 16; ++c) {
           if (c_beg + 16 * c < n_mma) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int t = c_beg + 16 * c + j;
-              const float v = h[16 * c + j];
+              const float h = v[16 * c + j];
               // 16-element block of h: lanes 0-15 or 16-31 of this warp. The
               // magnitudes' bit patterns order like the values.
-              uint32_t am = __float_as_uint(v) & 0x7FFFFFFFu;
+              uint32_t am = __float_as_uint(h) & 0x7FFFFFFFu;
 #pragma unroll
               for (int off = 1; off < 16; off <<= 1)
                 am = max(am, __shfl_xor_sync(0xffffffffu, am, off));
               const uint32_t s8 = cvt_e4m3(__fdividef(__uint_as_float(am), six_g));
               const float d = e4m3_to_f32(s8) * p.h_scale;
-              uint32_t code = cvt_e2m1(__fdividef(v, d));
+              uint32_t code = cvt_e2m1(__fdividef(h, d));
               code = s8 ? code : 0u;
               const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, 1);
               if (t < rows) {
@@ -417,26 +444,20 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
           }
         }
       } else {
-        const int64_t row0 = __ldg(p.offsets + e) + (int64_t)nb * kBN;
-        float* out = static_cast<float*>(p.out) + mb * kBM + r;
-        for (int c0 = 0; c0 < n_mma; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld16(tb + c0, v);
+        // y = acc x scale straight from TMEM; the second accumulator stage
+        // keeps the MMA warp busy meanwhile
+        const int64_t row0 = __ldg(p.offsets + e) + (int64_t)tt * TOK;
+        float* out = static_cast<float*>(p.out) + (row0 + c_beg) * p.out_ld + mb * kBM + r;
+        for (int c0 = 0; c0 < HALF && c_beg + c0 < n_mma; c0 += 16) {
+          uint32_t y[16];
+          tmem_ld16(tb + c_beg + c0, y);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (c0 + j < rows) out[(row0 + c0 + j) * p.out_ld] = __uint_as_float(v[j]) * p.acc_scale;
+            if (c_beg + c0 + j < rows) out[(c0 + j) * p.out_ld] = __uint_as_float(y[j]) * p.acc_scale;
         }
-      }
-      if (!GATEUP) {
         tc_fence_before();
-        mbar_arrive(&tempty[acc]);
-      }
-      if (C::kAccStages == 2) {
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-      } else {
-        acc_phase ^= 1u;
+        mbar_arrive(released);
       }
     }
   }
@@ -522,6 +543,7 @@ static Fp4Params base_params4(const beam_moe_cfg& c, const Fp4Layout& F, char* w
   p.counts = reinterpret_cast<const int32_t*>(ws + L.counts);
   p.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
   p.nb_off = reinterpret_cast<const int32_t*>(ws + L.nb_off);
+  p.tile_off = p.nb_off;
   p.E = c.n_experts;
   p.status = reinterpret_cast<unsigned*>(ws + L.status);
   p.I = c.inter;
@@ -561,6 +583,8 @@ cudaError_t launch_down_nvfp4(const beam_moe_cfg& c, const Fp4Layout& F,
   if (err != cudaSuccess) return err;
   err = encode_codes_map(&tx, ws + F.hq, (uint64_t)I / 2, (uint64_t)F.rows);
   if (err != cudaSuccess) return err;
+  if (Cfg4<false>::kTok == 256)  // token tiles of two 128-row blocks
+    p.tile_off = reinterpret_cast<const int32_t*>(ws + F.base.nb2_off);
   p.w_sf = w.w2_scales;
   p.x_sf = reinterpret_cast<const uint8_t*>(ws + F.hsf);
   p.out = ws + F.base.xp;
