@@ -166,14 +166,18 @@ __device__ __forceinline__ void decode_tile4(int tile, const Fp4Params& p, int& 
 
 template <bool GATEUP>
 struct Cfg4 {
-  // warp 0 TMA producer, warp 1 MMA issuer, then the epilogue warps. The
-  // gate/up epilogue (SwiGLU + NVFP4 quantisation of h) is the heavy one: two
-  // warps per TMEM lane quarter, each on half of the token columns, and its
-  // single accumulator is handed back as soon as it is read. The down
-  // epilogue only scales and stores y; it has one warp per lane quarter and a
-  // second accumulator stage instead.
+  // warp 0 TMA producer, warp 1 MMA issuer, warps 2-3 scale copiers, then the
+  // epilogue warps. The MMA issuer issues nothing but MMAs: a tcgen05.cp
+  // costs its issuing thread about as long as an MMA, so the scale copies
+  // run from two other warps and overlap the MMAs. The gate/up epilogue
+  // (SwiGLU + NVFP4 quantisation of h) is the heavy one: two warps per TMEM
+  // lane quarter, each on half of the token columns, and its single
+  // accumulator is handed back as soon as it is read. The down epilogue only
+  // scales and stores y; it has one warp per lane quarter and a second
+  // accumulator stage instead.
   static constexpr int kEpiWarps = GATEUP ? 8 : 4;
-  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kFirstEpiWarp = 4;
+  static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
   static constexpr int kNA = GATEUP ? 2 : 1;   // 128-row A tiles (gate and up, or down)
   static constexpr int kTok = 128;             // token rows per tile (MMA N)
   static constexpr int kTB = kTok / 128;       // 128-row token blocks per tile
@@ -182,16 +186,27 @@ struct Cfg4 {
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   static constexpr int kAccCols = kNA * kTok;  // FP32 accumulator columns per tile
   static constexpr int kAccStages = GATEUP ? 1 : 2;
-  // Scale columns per stage: 4 per 64-element chunk and 128-row block. They
-  // rotate over several buffers, so the copy for a stage never overwrites
-  // columns that MMAs of the previous stages may still read.
+  // Scale columns per stage: 4 per 64-element chunk and 128-row block. Stage
+  // i uses scale buffer i mod kSfBufs, rewritten only after the MMAs of stage
+  // i - kSfBufs completed. gate/up keeps two buffers so that 128 TMEM columns
+  // are left to park h (FP32, one column per token) between forming it and
+  // quantising it: the accumulator is then free for the next tile, and the
+  // quantisation runs from TMEM 16 columns at a time with few live registers.
   static constexpr int kSfColsA = 16 * kNA;
   static constexpr int kSfCols = kSfColsA + 16 * kTB;
-  static constexpr int kSfBufs = 4;
+  static constexpr int kSfBufs = GATEUP ? 2 : kStages;
+  static constexpr int kParkCols = GATEUP ? kTok : 0;
   static constexpr int kTmemCols = 512;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+  // gate/up: a 512-byte staging slice per epilogue warp gathers 16 tokens'
+  // code bytes (16 x 16) and scale pairs (16 x 2) into wide global stores
+  static constexpr int kStageOut = GATEUP ? 512 : 0;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256 + kEpiWarps * kStageOut;
+  static_assert((3 * kStages + 7) * 8 + 8 <= 256, "barrier area");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
   static constexpr int kColsPerWarp = kTok * 4 / kEpiWarps;  // token columns per epilogue warp
-  static_assert(kAccStages * kAccCols + kSfBufs * kSfCols <= kTmemCols, "TMEM overflow");
+  static_assert(kAccStages * kAccCols + kSfBufs * kSfCols + kParkCols <= kTmemCols,
+                "TMEM overflow");
+  static_assert(kSfBufs <= kStages, "scale buffers");
   static_assert(kStages >= 2, "pipeline too shallow");
   static_assert(kColsPerWarp <= 128, "epilogue registers");
 };
@@ -209,10 +224,11 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
   // stage: [A codes (x kNA)][B codes (x kTB)][A scales (x kNA)][B scales (x kTB)]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
   uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
+  uint64_t* sfready = empty + STAGES;  // the stage's scales are in TMEM
+  uint64_t* tfull = sfready + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = tempty + 2;  // [0] MMA issuer, [1] and [2] scale copiers
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -220,12 +236,13 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sfready[s], 2);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 32 * C::kEpiWarps);
     }
-    mbar_init(drain, 1);
+    for (int d = 0; d < 3; ++d) mbar_init(&drain[d], 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_w);
@@ -240,6 +257,7 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const uint32_t tsf = tmem_base + (uint32_t)(C::kAccStages * C::kAccCols);
+  const uint32_t tpark = tsf + (uint32_t)(C::kSfBufs * C::kSfCols);
   const int total = __ldg(p.tile_off + p.E) * p.n_mblk;
   const int sf_chunks = p.Kel / 64;  // scale atoms per 128-row block
 
@@ -319,29 +337,16 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
         const uint32_t d0 = tmem_base + (uint32_t)(acc * C::kAccCols);
         const uint32_t d1 = d0 + TOK;
         for (int kb = 0; kb < p.nk; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, kFlagMma)) {
+          // operands landed and their scales copied to this stage's columns
+          if (!mbar_wait(&sfready[stage], phase, abort_flag, p.status, kFlagMma)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sa = smem_addr(smem + stage * C::kStageBytes);
-          const uint32_t ssf = sa + (C::kNA + C::kTB) * kCodeTile;
           const uint32_t tsf_s = tsf + (uint32_t)(sfbuf * C::kSfCols);
           const uint32_t tsfb = tsf_s + C::kSfColsA;
           if (++sfbuf == C::kSfBufs) sfbuf = 0;
-          // Scale atoms of this stage into TMEM. Chunk j of the A tile(s) at
-          // columns 4j (gate or down) and 16 + 4j (up); chunk j of token block
-          // b at 4 (kTB j + b), so that a 256-row B operand finds rows
-          // 128-255 in the four columns after rows 0-127.
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tmem_cp_sf_atom(tsf_s + 4 * j, smem_desc_sf_atom(ssf + 512 * j));
-            if (GATEUP) tmem_cp_sf_atom(tsf_s + 16 + 4 * j, smem_desc_sf_atom(ssf + kSfStage + 512 * j));
-#pragma unroll
-            for (int b = 0; b < C::kTB; ++b)  // an absent second block copies stale bytes
-              tmem_cp_sf_atom(tsfb + 4 * (C::kTB * j + b),
-                              smem_desc_sf_atom(ssf + (C::kNA + b) * kSfStage + 512 * j));
-          }
           const uint64_t da0 = smem_desc_k_sw128(sa);
           const uint64_t da1 = smem_desc_k_sw128(sa + kCodeTile);
           const uint64_t db = smem_desc_k_sw128(sa + C::kNA * kCodeTile);
@@ -369,6 +374,55 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
       mbar_wait(drain, 0, nullptr, nullptr, 0u, 100000000ull);
     }
     __syncwarp();
+  } else if (warp < C::kFirstEpiWarp) {
+    if (lane == 0) {
+      // ------------------------------------------------------ scale copiers
+      // Warp 2 copies chunks 0-1 of every operand's scales, warp 3 chunks
+      // 2-3, into the stage's TMEM columns: chunk j of the A tile(s) at 4j
+      // (gate or down) and 16 + 4j (up), chunk j of token block b at
+      // kSfColsA + 4 (kTB j + b), so that a 256-row B operand would find rows
+      // 128-255 in the four columns after rows 0-127. Each commits to the
+      // stage's sfready barrier, which completes when both warps' copies have.
+      const int j0 = 2 * (warp - 2);
+      const int64_t ntiles = total > (int)blockIdx.x ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+      const int64_t nstages = ntiles * p.nk;
+      int stage = 0;
+      uint32_t phase = 0;
+      int sfbuf = 0;
+      for (int64_t i = 0; i < nstages; ++i) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, p.status, kFlagMma)) break;
+        if (C::kSfBufs < STAGES && i >= C::kSfBufs) {
+          // the MMAs of stage i - kSfBufs, which read this buffer, are done
+          const int64_t k = i - C::kSfBufs;
+          if (!mbar_wait(&empty[k % STAGES], (uint32_t)((k / STAGES) & 1), abort_flag, p.status,
+                         kFlagMma))
+            break;
+        }
+        tc_fence_after();
+        const uint32_t ssf = smem_addr(smem + stage * C::kStageBytes) + (C::kNA + C::kTB) * kCodeTile;
+        const uint32_t tsf_s = tsf + (uint32_t)(sfbuf * C::kSfCols);
+        if (++sfbuf == C::kSfBufs) sfbuf = 0;
+        const uint32_t tsfb = tsf_s + C::kSfColsA;
+#pragma unroll
+        for (int j = j0; j < j0 + 2; ++j) {
+          tmem_cp_sf_atom(tsf_s + 4 * j, smem_desc_sf_atom(ssf + 512 * j));
+          if (GATEUP) tmem_cp_sf_atom(tsf_s + 16 + 4 * j, smem_desc_sf_atom(ssf + kSfStage + 512 * j));
+#pragma unroll
+          for (int b = 0; b < C::kTB; ++b)  // an absent second block copies stale bytes
+            tmem_cp_sf_atom(tsfb + 4 * (C::kTB * j + b),
+                            smem_desc_sf_atom(ssf + (C::kNA + b) * kSfStage + 512 * j));
+        }
+        umma_commit(&sfready[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      uint64_t* own = &drain[1 + (warp - 2)];
+      umma_commit(own);  // this warp's copies are done before TMEM is freed
+      mbar_wait(own, 0, nullptr, nullptr, 0u, 100000000ull);
+    }
+    __syncwarp();
   } else {
     // -------------------------------------------------------------- epilogue
     // Each warp owns TMEM lane quarter q (32 weight rows) and token columns
@@ -376,7 +430,7 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
     constexpr int HALF = C::kColsPerWarp;
     const int q = warp & 3;
     const int r = q * 32 + lane;  // weight row inside the 128-row tile
-    const int c_beg = ((warp - 2) >> 2) * HALF;
+    const int c_beg = ((warp - C::kFirstEpiWarp) >> 2) * HALF;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -393,54 +447,79 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
         acc_phase ^= 1u;
       }
       if (GATEUP) {
-        // h = silu(g) u into registers, then TMEM goes back to the MMA warp
-        float v[HALF];
+        // h = silu(g) u, parked in this warp's TMEM columns; then the
+        // accumulator goes back to the MMA warp
+        const uint32_t tp = tpark + ((uint32_t)(q * 32) << 16) + (uint32_t)c_beg;
 #pragma unroll
         for (int c = 0; c < HALF / 16; ++c) {
           if (c_beg + 16 * c < n_mma) {  // warp-uniform
-            uint32_t g[16], u[16];
+            uint32_t g[16], u[16], hb[16];
             tmem_ld16(tb + c_beg + 16 * c, g);
             tmem_ld16(tb + TOK + c_beg + 16 * c, u);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              v[16 * c + j] = gg::silu_mul(__uint_as_float(g[j]) * p.acc_scale,
-                                           __uint_as_float(u[j]) * p.acc_scale);
+              hb[j] = __float_as_uint(gg::silu_mul(__uint_as_float(g[j]) * p.acc_scale,
+                                                   __uint_as_float(u[j]) * p.acc_scale));
+            tmem_st16(tp + 16 * c, hb);
           }
         }
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(released);
 
-        const int idx = mb * kBM + r;  // intermediate index of this lane
+        // This warp's 32 intermediate indices start at i0: 16 code bytes per
+        // token, and 2 scale bytes (blocks i0/16 and i0/16 + 1, adjacent in
+        // the atom layout) per token.
+        const int i0 = mb * kBM + q * 32;
         const int64_t qrow0 = (int64_t)(__ldg(p.nb_off + e) + tt) * kBN;  // 128-row aligned
-        uint8_t* hq = static_cast<uint8_t*>(p.out) + qrow0 * p.out_ld + idx / 2;
-        // scale byte of (row qrow0 + t, block idx / 16) in the atom layout
+        uint8_t* hq = static_cast<uint8_t*>(p.out) + qrow0 * p.out_ld + i0 / 2;
         uint8_t* hsf = p.out_sf +
-                       ((qrow0 >> 7) * (p.I >> 6) + (idx >> 6)) * 512 + ((idx >> 4) & 3);
+                       ((qrow0 >> 7) * (p.I >> 6) + (i0 >> 6)) * 512 + ((i0 >> 4) & 3);
+        uint8_t* so = smem + STAGES * C::kStageBytes + 256 +
+                      (warp - C::kFirstEpiWarp) * C::kStageOut;  // [16 tokens][16 B], [16][2 B]
         const float six_g = 6.0f * p.h_scale;
-#pragma unroll
+#pragma unroll 2
         for (int c = 0; c < HALF / 16; ++c) {
           if (c_beg + 16 * c < n_mma) {
+            uint32_t hb[16];
+            tmem_ld16(tp + 16 * c, hb);
+            tmem_ld_wait();
+            // Codes and scales of 16 tokens first, with no control flow, so
+            // that their shuffle and conversion chains overlap; then the
+            // stores. Tokens from `rows` up to the 16-row boundary land in
+            // the padding of this expert's 128-row segment, which no
+            // consumer reads, so they need no guard.
+            uint32_t packed[16], scale[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const int t = c_beg + 16 * c + j;
-              const float h = v[16 * c + j];
+              const float h = __uint_as_float(hb[j]);
               // 16-element block of h: lanes 0-15 or 16-31 of this warp. The
               // magnitudes' bit patterns order like the values.
-              uint32_t am = __float_as_uint(h) & 0x7FFFFFFFu;
+              uint32_t am = hb[j] & 0x7FFFFFFFu;
 #pragma unroll
               for (int off = 1; off < 16; off <<= 1)
                 am = max(am, __shfl_xor_sync(0xffffffffu, am, off));
               const uint32_t s8 = cvt_e4m3(__fdividef(__uint_as_float(am), six_g));
               const float d = e4m3_to_f32(s8) * p.h_scale;
-              uint32_t code = cvt_e2m1(__fdividef(h, d));
-              code = s8 ? code : 0u;
-              const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, 1);
-              if (t < rows) {
-                if ((lane & 1) == 0) hq[t * p.out_ld] = (uint8_t)(code | (partner << 4));
-                if ((lane & 15) == 0) hsf[(t & 31) * 16 + (t >> 5) * 4] = (uint8_t)s8;
-              }
+              const uint32_t code = s8 ? cvt_e2m1(__fdividef(h, d)) : 0u;
+              packed[j] = code | (__shfl_xor_sync(0xffffffffu, code, 1) << 4);
+              scale[j] = s8;
             }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              if ((lane & 1) == 0) so[16 * j + (lane >> 1)] = (uint8_t)packed[j];
+              if ((lane & 15) == 0) so[256 + 2 * j + (lane >> 4)] = (uint8_t)scale[j];
+            }
+            __syncwarp();
+            if (lane < 16) {  // token t = c_beg + 16 c + lane
+              const int t = c_beg + 16 * c + lane;
+              *reinterpret_cast<uint4*>(hq + t * p.out_ld) =
+                  *reinterpret_cast<const uint4*>(so + 16 * lane);
+              *reinterpret_cast<uint16_t*>(hsf + (t & 31) * 16 + (t >> 5) * 4) =
+                  *reinterpret_cast<const uint16_t*>(so + 256 + 2 * lane);
+            }
+            __syncwarp();
           }
         }
       } else {

@@ -3,6 +3,7 @@
 // MMA, and the E4M3 / E2M1 conversions. Encodings follow the PTX ISA.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "sm100.cuh"
@@ -59,6 +60,20 @@ __device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t adesc, uint6
       : "memory");
 }
 
+// TMEM store, 32 lanes x 32 bits, 16 consecutive columns (this warp's lane quarter).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // FP32 -> E4M3 byte (nearest, ties to even, saturating at 448).
 __device__ __forceinline__ uint32_t cvt_e4m3(float v) {
   uint16_t r;
@@ -79,8 +94,11 @@ __device__ __forceinline__ uint32_t cvt_e2m1(float v) {
 
 // E4M3 byte (non-negative, finite) -> FP32, exact.
 __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
-  const uint32_t E = (b >> 3) & 15u, f = b & 7u;
-  return E ? __uint_as_float(((E + 120u) << 23) | (f << 20)) : (float)f * 0.001953125f;
+  // hardware E4M3 -> F16 conversion of the byte pair (b, 0); the zero byte
+  // converts to +0, so OR-ing the halves picks b's value in either order
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(b & 0xFFu)));
+  return __half2float(__ushort_as_half((uint16_t)((h2 | (h2 >> 16)) & 0xFFFFu)));
 }
 
 }  // namespace beam
