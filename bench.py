@@ -48,7 +48,10 @@ METRIC = "MoE-block tokens/s; achieved TFLOP/s or HBM GB/s as % of B200 roofline
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 STAGES = ("router_gemm", "router_topk", "scan", "permute", "gateup_gemm", "down_gemm", "combine")
-KERNELS_PER_STEP = 7
+# router weight split, router GEMM, top-k, scan, permute, gate/up, down, combine;
+# replayed routes skip the first two and add one kernel that copies the routes in
+KERNELS_PER_STEP = 8
+KERNELS_PER_REPLAY_STEP = 6
 GEMM_SOURCES = ("sparse_moe_layer_beam_b200/csrc/grouped_gemm.cu",
                 "sparse_moe_layer_beam_b200/csrc/sm100.cuh")
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the gate/up
@@ -437,7 +440,8 @@ def run_ours(args, wl):
         "stages_ms": None if args.replay else stage_mean,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * wl.H * 2,
                 "d2h_bytes_per_step": wl.T * wl.H * 2},
-        "gpu_launches": (KERNELS_PER_STEP - (1 if args.replay else 0)) * args.steps,
+        "gpu_launches": (KERNELS_PER_REPLAY_STEP if args.replay else KERNELS_PER_STEP)
+        * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -46,14 +46,21 @@ static int pick_bn(int64_t T, int K, int E) {
   return 256;
 }
 
-Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms) {
+Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool tc_router) {
   Layout L;
   memset(&L, 0, sizeof(L));
   const int E = c.n_experts, K = c.top_k, H = c.hidden, I = c.inter;
   L.T = T;
   L.A = T * K;
   L.nchunks = (int)((T + kChunk - 1) / kChunk);
-  L.split_k = router_split_k(T, H, E, sms);
+  L.router_tc = (tc_router && router_tc_supported(c)) ? 1 : 0;
+  if (L.router_tc) {
+    const int nkb = H / 64;
+    L.router_kper = router_tc_kper(T, H, E, sms);
+    L.split_k = (nkb + L.router_kper - 1) / L.router_kper;
+  } else {
+    L.split_k = router_split_k(T, H, E, sms);
+  }
   L.bn = pick_bn(T, K, E);
   // CTA pairs halve the token-row bytes each SM reads per weight byte and
   // double-buffer the accumulator. That pays once experts average 64 rows or
@@ -81,6 +88,7 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms) {
   L.chunk_cnt = take(sizeof(int32_t) * (size_t)L.nchunks * E, 256);
   L.chunk_mask = take(sizeof(uint32_t) * (size_t)L.nchunks * E * kChunkWords, 256);
   L.logits = take(sizeof(float) * (size_t)L.split_k * T * E, 256);
+  L.w3 = L.router_tc ? take(2 * 3 * (size_t)E * H, 1024) : 0;
   L.route_end = align_up(o, 256);
   // permuted rows (bf16) during gate/up, then the down output y (fp32)
   L.xp = take(4 * (size_t)L.A * H, 1024);

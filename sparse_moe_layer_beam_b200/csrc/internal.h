@@ -30,7 +30,9 @@ constexpr uint32_t kFlagBadExpert = 0x100;
 struct Layout {
   int64_t T, A;     // tokens, assignments (T * K)
   int nchunks;      // ceil(T / kChunk)
-  int split_k;      // router split-K factor
+  int split_k;      // router split-K factor (slices of partial logits)
+  int router_tc;    // 1: router GEMM on tensor cores (router_tc.cu), 0: CUDA cores
+  int router_kper;  // tensor-core router: K blocks of 64 per split
   int bn;           // token tile of the grouped GEMMs
   int pair_gateup; // 1: gate/up grouped GEMM on CTA pairs
   int pair_down;   // 1: down grouped GEMM on CTA pairs
@@ -45,13 +47,15 @@ struct Layout {
   size_t chunk_cnt; // int32[nchunks * E] first row of each (chunk, expert)
   size_t chunk_mask;// uint32[nchunks * E * kChunkWords]
   size_t logits;    // float[split_k * T * E] partial router logits
+  size_t w3;        // bf16[3][E][H] exact three-way split of the router weights
   size_t route_end; // bytes needed by the routing op
   size_t xp;        // bf16[A * H] permuted rows; reused for the down output y, fp32[A * H]
   size_t h;         // bf16[A * I] SwiGLU activations
   size_t total;     // bytes needed by the forward op
 };
 
-Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms);
+// tc_router = false keeps the router on CUDA cores (no weight planes needed).
+Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool tc_router = true);
 
 // NVFP4 path: the routing layout (token tiles of 128 rows, expert segments
 // padded to them) plus quantised activations and their scales.
@@ -67,8 +71,14 @@ Fp4Layout make_layout_nvfp4(const beam_moe_cfg& c, int64_t T, int sms);
 bool nvfp4_supported(const beam_moe_cfg& c);
 
 // ---- launchers (each enqueues on `st`, returns cudaGetLastError()) --------
+// Router GEMM into the partial logits: the tensor-core kernel when
+// L.router_tc, else the CUDA-core kernel. Either clears the dispatch bits.
 cudaError_t launch_router_logits(const beam_moe_cfg& c, const Layout& L, const uint16_t* x,
                                  const float* w_router, char* ws, cudaStream_t st);
+cudaError_t launch_router_tc(const beam_moe_cfg& c, const Layout& L, const uint16_t* x,
+                             const float* w_router, char* ws, cudaStream_t st);
+bool router_tc_supported(const beam_moe_cfg& c);
+int router_tc_kper(int64_t T, int H, int E, int sms);
 cudaError_t launch_router_topk(const beam_moe_cfg& c, const Layout& L, const float* bias,
                                char* ws, cudaStream_t st);
 cudaError_t launch_routes_given(const beam_moe_cfg& c, const Layout& L, const int32_t* ids,

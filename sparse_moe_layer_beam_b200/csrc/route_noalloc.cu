@@ -57,10 +57,10 @@ extern "C" BEAM_MOE_API beam_moe_status beam_moe_route_noalloc(
 
   // Fewer router splits when the split partial sums would not fit.
   int sms = beam::device_sm_count();
-  beam::Layout L = beam::make_layout(*cfg, T, sms);
+  beam::Layout L = beam::make_layout(*cfg, T, sms, false);
   while (L.route_end > kScratchBytes && sms > 1) {
     sms /= 2;
-    L = beam::make_layout(*cfg, T, sms);
+    L = beam::make_layout(*cfg, T, sms, false);
   }
   if (L.route_end > kScratchBytes) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
 

@@ -348,6 +348,7 @@ int router_split_k(int64_t T, int H, int E, int sms) {
 
 cudaError_t launch_router_logits(const beam_moe_cfg& c, const Layout& L, const uint16_t* x,
                                  const float* w_router, char* ws, cudaStream_t st) {
+  if (L.router_tc) return launch_router_tc(c, L, x, w_router, ws, st);
   const int H = c.hidden, E = c.n_experts;
   dim3 grid((unsigned)((L.T + kRBM - 1) / kRBM), (unsigned)((E + kRBE - 1) / kRBE),
             (unsigned)L.split_k);
