@@ -357,9 +357,28 @@ def run_ours(args, wl):
     if flags:
         raise SystemExit(f"device status flags {flags:#x} in the timed region")
 
-    # end to end through the public call with host buffers: pinned x in, out back
+    # End to end with host buffers: pinned x in, out back. The forward goes
+    # through beam_moe_forward_host (chunked, copies overlapped with compute);
+    # replayed routes have no host-buffer entry point, so that line copies
+    # around beam_moe_forward_routed.
     x_host = x.cpu().pin_memory()
     out_host = torch.empty_like(out, device="cpu").pin_memory()
+    ws_h = None
+    if not args.replay:
+        op_h = bm.OP_FORWARD_NVFP4_HOST if nvfp4 else bm.OP_FORWARD_HOST
+        ws_h = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T, op_h), dtype=torch.uint8,
+                           device=dev)
+
+    def e2e_step():
+        if nvfp4:
+            bm.beam_moe_forward_nvfp4_host(cfg, x_host, wr, b, experts, out_host, ws_h, stream=st)
+        elif not args.replay:
+            bm.beam_moe_forward_host(cfg, x_host, wr, b, w13, w2, out_host, ws_h, stream=st)
+        else:
+            x.copy_(x_host, non_blocking=True)
+            step()
+            out_host.copy_(out, non_blocking=True)
+
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     for i in range(args.warmup + args.steps):
@@ -367,9 +386,7 @@ def run_ours(args, wl):
         j = i - args.warmup
         if j >= 0:
             e2e_ev[j][0].record(stream)
-        x.copy_(x_host, non_blocking=True)
-        step()
-        out_host.copy_(out, non_blocking=True)
+        e2e_step()
         if j >= 0:
             e2e_ev[j][1].record(stream)
     torch.cuda.synchronize()
@@ -439,7 +456,10 @@ def run_ours(args, wl):
                   "touched_experts": alg["touched_experts"]},
         "stages_ms": None if args.replay else stage_mean,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * wl.H * 2,
-                "d2h_bytes_per_step": wl.T * wl.H * 2},
+                "d2h_bytes_per_step": wl.T * wl.H * 2,
+                "call": ("copies around beam_moe_forward_routed" if args.replay else
+                         ("beam_moe_forward_nvfp4_host" if nvfp4 else "beam_moe_forward_host")
+                         + " (chunked from 16384 tokens, copies overlapped)")},
         "gpu_launches": (KERNELS_PER_REPLAY_STEP if args.replay else KERNELS_PER_STEP)
         * args.steps,
         "clocks": clk,

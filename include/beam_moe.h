@@ -77,6 +77,8 @@ typedef enum beam_moe_op {
   BEAM_MOE_OP_ROUTE = 0,         /* beam_moe_route                            */
   BEAM_MOE_OP_FORWARD = 1,       /* beam_moe_forward, beam_moe_forward_routed */
   BEAM_MOE_OP_FORWARD_NVFP4 = 2, /* beam_moe_forward_nvfp4                    */
+  BEAM_MOE_OP_FORWARD_HOST = 3,  /* beam_moe_forward_host                      */
+  BEAM_MOE_OP_FORWARD_NVFP4_HOST = 4, /* beam_moe_forward_nvfp4_host          */
 } beam_moe_op;
 
 /* Bytes of workspace the operation needs for T tokens (a pure host function). */
@@ -205,6 +207,39 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_nvfp4(const beam_moe_cfg* cfg, int
                                                     uint16_t* out, int32_t* topk_ids,
                                                     float* topk_w, int32_t* expert_counts,
                                                     void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The block forward on activations in HOST memory, the call a serving loop
+ * makes with a batch it holds on the host. x_host [T][H] bf16 and out_host
+ * [T][H] bf16 are host buffers (page-locked, or the copies cannot overlap);
+ * w_router, bias, w13, w2 and ws are device memory as for beam_moe_forward.
+ * The result equals beam_moe_forward's for the same tokens. Batches of at
+ * least 2 * BEAM_MOE_HOST_CHUNK tokens run in chunks of that many tokens
+ * (bf16 batches of at least 8 * BEAM_MOE_HOST_CHUNK in chunks twice that
+ * size, so that each chunk's GEMMs stay compute-bound): the host-to-device
+ * copy of chunk i + 1 and the device-to-host copy of chunk i - 1 run on two
+ * copy streams the call creates, while chunk i computes on `stream`; smaller
+ * batches run as one chunk on `stream`. The call is
+ * stream-ordered: once `stream` has passed it, out_host holds the result.
+ * Each chunk is routed on its own, so the router's split of H (and with it
+ * the summation order of the FP32 logits) follows the chunk size.
+ * Workspace: BEAM_MOE_OP_FORWARD_HOST bytes (the forward workspace of one
+ * chunk plus two device staging buffers each for x and out). Calls that
+ * share a workspace must not overlap.
+ */
+#define BEAM_MOE_HOST_CHUNK 8192
+BEAM_MOE_API beam_moe_status beam_moe_forward_host(const beam_moe_cfg* cfg, int64_t T,
+                                                   const uint16_t* x_host, const float* w_router,
+                                                   const float* bias, const uint16_t* w13,
+                                                   const uint16_t* w2, uint16_t* out_host,
+                                                   void* ws, size_t ws_bytes, void* stream);
+
+/* The same with NVFP4 experts (beam_moe_forward_nvfp4 per chunk).
+ * Workspace: BEAM_MOE_OP_FORWARD_NVFP4_HOST bytes. */
+BEAM_MOE_API beam_moe_status beam_moe_forward_nvfp4_host(
+    const beam_moe_cfg* cfg, int64_t T, const uint16_t* x_host, const float* w_router,
+    const float* bias, const beam_moe_nvfp4_experts* experts, uint16_t* out_host, void* ws,
+    size_t ws_bytes, void* stream);
 
 /*
  * Quantise `rows` rows of K fp32 values (device, K a multiple of 16) to

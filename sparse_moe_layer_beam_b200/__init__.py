@@ -17,7 +17,9 @@ import os
 __all__ = ["BeamMoeCfg", "BeamMoeError", "Trace", "OP_ROUTE", "OP_FORWARD", "N_STAGES",
            "STAGE_NAMES", "lib", "beam_cfg", "beam_moe_workspace_size", "beam_moe_route",
            "beam_moe_route_noalloc", "BeamMoeNvfp4Experts", "OP_FORWARD_NVFP4", "nvfp4_experts",
-           "beam_moe_forward_nvfp4", "beam_moe_nvfp4_quantize",
+           "beam_moe_forward_nvfp4", "beam_moe_nvfp4_quantize", "OP_FORWARD_HOST",
+           "OP_FORWARD_NVFP4_HOST", "HOST_CHUNK", "beam_moe_forward_host",
+           "beam_moe_forward_nvfp4_host",
            "beam_moe_forward", "beam_moe_forward_routed", "beam_moe_forward_traced",
            "beam_moe_check"]
 
@@ -27,6 +29,9 @@ LIB_PATH = os.path.join(_HERE, "libbeam_moe.so")
 OP_ROUTE = 0
 OP_FORWARD = 1
 OP_FORWARD_NVFP4 = 2
+OP_FORWARD_HOST = 3
+OP_FORWARD_NVFP4_HOST = 4
+HOST_CHUNK = 8192
 N_STAGES = 7
 STAGE_NAMES = ("router_gemm", "router_topk", "scan", "permute", "gateup_gemm", "down_gemm",
                "combine")
@@ -73,6 +78,11 @@ _SIGS = {
     "beam_moe_forward_nvfp4_traced": [_CFG, ctypes.c_int64, _P, _P, _P,
                                       ctypes.POINTER(BeamMoeNvfp4Experts), _P, _P, _P, _P, _P,
                                       ctypes.c_size_t, _P, _P],
+    "beam_moe_forward_host": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                              _P],
+    "beam_moe_forward_nvfp4_host": [_CFG, ctypes.c_int64, _P, _P, _P,
+                                    ctypes.POINTER(BeamMoeNvfp4Experts), _P, _P, ctypes.c_size_t,
+                                    _P],
     "beam_moe_nvfp4_quantize": [ctypes.c_int64, ctypes.c_int64, _P, ctypes.c_float, _P, _P, _P],
     "beam_moe_trace_create": [ctypes.c_int32, ctypes.POINTER(_P)],
     "beam_moe_trace_destroy": [_P],
@@ -180,6 +190,24 @@ def nvfp4_experts(w13_codes, w13_scales, w2_codes, w2_scales, w13_scale, w2_scal
                   h_scale):
     return BeamMoeNvfp4Experts(_ptr(w13_codes), _ptr(w13_scales), _ptr(w2_codes),
                                _ptr(w2_scales), w13_scale, w2_scale, x_scale, h_scale)
+
+
+def beam_moe_forward_host(cfg, x_host, w_router, bias, w13, w2, out_host, ws, stream=None):
+    """Forward on host buffers (x_host, out_host: CPU tensors, pinned for overlap)."""
+    T = x_host.shape[0]
+    _check(lib().beam_moe_forward_host(ctypes.byref(cfg), T, _ptr(x_host), _ptr(w_router),
+                                       _ptr(bias), _ptr(w13), _ptr(w2), _ptr(out_host), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)),
+           "beam_moe_forward_host")
+
+
+def beam_moe_forward_nvfp4_host(cfg, x_host, w_router, bias, experts, out_host, ws, stream=None):
+    T = x_host.shape[0]
+    _check(lib().beam_moe_forward_nvfp4_host(ctypes.byref(cfg), T, _ptr(x_host), _ptr(w_router),
+                                             _ptr(bias), ctypes.byref(experts), _ptr(out_host),
+                                             _ptr(ws), ws.numel() * ws.element_size(),
+                                             _stream(stream)),
+           "beam_moe_forward_nvfp4_host")
 
 
 def beam_moe_forward_nvfp4(cfg, x, w_router, bias, experts, out, ws, topk_ids=None, topk_w=None,

@@ -366,9 +366,159 @@ beam_moe_status forward_nvfp4_impl(const beam_moe_cfg* cfg, int64_t T, const uin
   return BEAM_MOE_OK;
 }
 
+// ------------------------------------------------------------ host buffers
+// Chunking of a forward on host buffers: chunks of BEAM_MOE_HOST_CHUNK tokens
+// once there are at least two, else one chunk; bf16 batches of at least
+// 8 x BEAM_MOE_HOST_CHUNK tokens take chunks twice as large, because every
+// chunk streams all touched experts once (20 GB in bf16) and at 8192 tokens
+// that costs about 13 % of the compute. The chunk's forward workspace is
+// sized for the larger of the full and the last chunk (the router's split of
+// H, and with it the partial-logit buffer, is not monotone in T).
+struct HostPlan {
+  int64_t chunk, n_chunks;
+  size_t fwd_bytes;  // forward workspace of one chunk
+  size_t buf_bytes;  // one staging buffer: chunk x H bf16
+  int n_bufs;        // staging buffers per direction
+  size_t total;
+};
+
+beam_moe_status host_plan(const beam_moe_cfg* cfg, int64_t T, beam_moe_op fwd_op, HostPlan* hp) {
+  const int64_t c = BEAM_MOE_HOST_CHUNK;
+  hp->chunk = T < 2 * c ? T : ((fwd_op == BEAM_MOE_OP_FORWARD && T >= 8 * c) ? 2 * c : c);
+  hp->n_chunks = (T + hp->chunk - 1) / hp->chunk;
+  const int64_t last = T - (hp->n_chunks - 1) * hp->chunk;
+  size_t a = 0, b = 0;
+  BEAM_TRY(beam_moe_workspace_size(cfg, hp->chunk, fwd_op, &a));
+  BEAM_TRY(beam_moe_workspace_size(cfg, last, fwd_op, &b));
+  hp->fwd_bytes = beam::align_up(a > b ? a : b, 1024);
+  hp->buf_bytes = beam::align_up((size_t)hp->chunk * cfg->hidden * 2, 1024);
+  hp->n_bufs = hp->n_chunks > 1 ? 2 : 1;
+  hp->total = hp->fwd_bytes + 2 * (size_t)hp->n_bufs * hp->buf_bytes;
+  return BEAM_MOE_OK;
+}
+
+// Runs forward(Tc, x_dev, out_dev, fwd_ws, fwd_bytes, stream) per chunk. With
+// several chunks, a chunk's upload waits until the forward two chunks back
+// has read its staging buffer, its forward waits for its upload and for the
+// download two chunks back, and its download waits for its forward. The
+// caller's stream finally waits for the last download.
+template <class Fwd>
+beam_moe_status host_pipeline(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x_host,
+                              uint16_t* out_host, char* ws, const HostPlan& hp,
+                              cudaStream_t st, Fwd forward) {
+  const int64_t H = cfg->hidden;
+  uint16_t* xb[2];
+  uint16_t* ob[2];
+  for (int b = 0; b < hp.n_bufs; ++b) {
+    xb[b] = reinterpret_cast<uint16_t*>(ws + hp.fwd_bytes + b * hp.buf_bytes);
+    ob[b] = reinterpret_cast<uint16_t*>(ws + hp.fwd_bytes + (hp.n_bufs + b) * hp.buf_bytes);
+  }
+  if (hp.n_chunks == 1) {
+    BEAM_CUDA(cudaMemcpyAsync(xb[0], x_host, (size_t)T * H * 2, cudaMemcpyHostToDevice, st));
+    BEAM_TRY(forward(T, xb[0], ob[0], ws, hp.fwd_bytes, st));
+    BEAM_CUDA(cudaMemcpyAsync(out_host, ob[0], (size_t)T * H * 2, cudaMemcpyDeviceToHost, st));
+    return BEAM_MOE_OK;
+  }
+  // streams and events of this call; their destruction is deferred by the
+  // runtime until the work that uses them has completed
+  struct Res {
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t ev[8] = {};
+    ~Res() {
+      for (cudaEvent_t e : ev)
+        if (e) cudaEventDestroy(e);
+      if (up) cudaStreamDestroy(up);
+      if (down) cudaStreamDestroy(down);
+    }
+  } r;
+  BEAM_CUDA(cudaStreamCreateWithFlags(&r.up, cudaStreamNonBlocking));
+  BEAM_CUDA(cudaStreamCreateWithFlags(&r.down, cudaStreamNonBlocking));
+  for (cudaEvent_t& e : r.ev) BEAM_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  cudaEvent_t start = r.ev[0], done = r.ev[1];
+  cudaEvent_t* uploaded = r.ev + 2;    // [2] staged x of a chunk is on the device
+  cudaEvent_t* computed = r.ev + 4;    // [2] a chunk's forward has finished
+  cudaEvent_t* downloaded = r.ev + 6;  // [2] a chunk's out has reached the host
+  BEAM_CUDA(cudaEventRecord(start, st));  // the copies start after earlier work on st
+  BEAM_CUDA(cudaStreamWaitEvent(r.up, start, 0));
+  BEAM_CUDA(cudaStreamWaitEvent(r.down, start, 0));
+  for (int64_t i = 0; i < hp.n_chunks; ++i) {
+    const int b = (int)(i & 1);
+    const int64_t t0 = i * hp.chunk;
+    const int64_t tc = (T - t0) < hp.chunk ? (T - t0) : hp.chunk;
+    const size_t bytes = (size_t)tc * H * 2;
+    if (i >= 2) BEAM_CUDA(cudaStreamWaitEvent(r.up, computed[b], 0));
+    BEAM_CUDA(cudaMemcpyAsync(xb[b], x_host + t0 * H, bytes, cudaMemcpyHostToDevice, r.up));
+    BEAM_CUDA(cudaEventRecord(uploaded[b], r.up));
+    BEAM_CUDA(cudaStreamWaitEvent(st, uploaded[b], 0));
+    if (i >= 2) BEAM_CUDA(cudaStreamWaitEvent(st, downloaded[b], 0));
+    BEAM_TRY(forward(tc, xb[b], ob[b], ws, hp.fwd_bytes, st));
+    BEAM_CUDA(cudaEventRecord(computed[b], st));
+    BEAM_CUDA(cudaStreamWaitEvent(r.down, computed[b], 0));
+    BEAM_CUDA(cudaMemcpyAsync(out_host + t0 * H, ob[b], bytes, cudaMemcpyDeviceToHost, r.down));
+    BEAM_CUDA(cudaEventRecord(downloaded[b], r.down));
+  }
+  BEAM_CUDA(cudaEventRecord(done, r.down));
+  BEAM_CUDA(cudaStreamWaitEvent(st, done, 0));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status host_checks(const beam_moe_cfg* cfg, int64_t T, const void* x_host,
+                            const void* out_host, void* ws, size_t ws_bytes, beam_moe_op op,
+                            HostPlan* hp) {
+  BEAM_TRY(check_cfg(cfg));
+  BEAM_TRY(check_T(cfg, T));
+  if (T == 0) return BEAM_MOE_OK;
+  if (!x_host || !out_host || !ws) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return BEAM_MOE_ERR_ALIGNMENT;
+  BEAM_TRY(host_plan(cfg, T,
+                     op == BEAM_MOE_OP_FORWARD_HOST ? BEAM_MOE_OP_FORWARD
+                                                    : BEAM_MOE_OP_FORWARD_NVFP4,
+                     hp));
+  if (ws_bytes < hp->total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+  return BEAM_MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+beam_moe_status beam_moe_forward_host(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x_host,
+                                      const float* w_router, const float* bias,
+                                      const uint16_t* w13, const uint16_t* w2, uint16_t* out_host,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  HostPlan hp;
+  BEAM_TRY(host_checks(cfg, T, x_host, out_host, ws, ws_bytes, BEAM_MOE_OP_FORWARD_HOST, &hp));
+  if (T == 0) return BEAM_MOE_OK;
+  BEAM_TRY(check_ptrs({w_router, w13, w2}, {bias}));
+  return host_pipeline(
+      cfg, T, x_host, out_host, static_cast<char*>(ws), hp,
+      reinterpret_cast<cudaStream_t>(stream),
+      [&](int64_t tc, const uint16_t* xd, uint16_t* od, char* fws, size_t fb, cudaStream_t s) {
+        return forward_impl(cfg, tc, xd, w_router, bias, w13, w2, od, nullptr, nullptr, nullptr,
+                            fws, fb, s, nullptr);
+      });
+}
+
+beam_moe_status beam_moe_forward_nvfp4_host(const beam_moe_cfg* cfg, int64_t T,
+                                            const uint16_t* x_host, const float* w_router,
+                                            const float* bias,
+                                            const beam_moe_nvfp4_experts* experts,
+                                            uint16_t* out_host, void* ws, size_t ws_bytes,
+                                            void* stream) {
+  if (cfg && !beam::nvfp4_supported(*cfg)) return BEAM_MOE_ERR_UNSUPPORTED_SHAPE;
+  HostPlan hp;
+  BEAM_TRY(
+      host_checks(cfg, T, x_host, out_host, ws, ws_bytes, BEAM_MOE_OP_FORWARD_NVFP4_HOST, &hp));
+  if (T == 0) return BEAM_MOE_OK;
+  if (!experts) return BEAM_MOE_ERR_INVALID_ARG;
+  return host_pipeline(
+      cfg, T, x_host, out_host, static_cast<char*>(ws), hp,
+      reinterpret_cast<cudaStream_t>(stream),
+      [&](int64_t tc, const uint16_t* xd, uint16_t* od, char* fws, size_t fb, cudaStream_t s) {
+        return forward_nvfp4_impl(cfg, tc, xd, w_router, bias, experts, od, nullptr, nullptr,
+                                  nullptr, fws, fb, s, nullptr);
+      });
+}
 
 beam_moe_status beam_moe_forward_nvfp4(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
                                        const float* w_router, const float* bias,
@@ -407,12 +557,23 @@ beam_moe_status beam_moe_workspace_size(const beam_moe_cfg* cfg, int64_t T, beam
   BEAM_TRY(check_cfg(cfg));
   BEAM_TRY(check_T(cfg, T));
   if (!bytes || (op != BEAM_MOE_OP_ROUTE && op != BEAM_MOE_OP_FORWARD &&
-                 op != BEAM_MOE_OP_FORWARD_NVFP4))
+                 op != BEAM_MOE_OP_FORWARD_NVFP4 && op != BEAM_MOE_OP_FORWARD_HOST &&
+                 op != BEAM_MOE_OP_FORWARD_NVFP4_HOST))
     return BEAM_MOE_ERR_INVALID_ARG;
-  if (op == BEAM_MOE_OP_FORWARD_NVFP4 && !beam::nvfp4_supported(*cfg))
+  if ((op == BEAM_MOE_OP_FORWARD_NVFP4 || op == BEAM_MOE_OP_FORWARD_NVFP4_HOST) &&
+      !beam::nvfp4_supported(*cfg))
     return BEAM_MOE_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) {
     *bytes = 0;
+    return BEAM_MOE_OK;
+  }
+  if (op == BEAM_MOE_OP_FORWARD_HOST || op == BEAM_MOE_OP_FORWARD_NVFP4_HOST) {
+    HostPlan hp;
+    BEAM_TRY(host_plan(cfg, T,
+                       op == BEAM_MOE_OP_FORWARD_HOST ? BEAM_MOE_OP_FORWARD
+                                                      : BEAM_MOE_OP_FORWARD_NVFP4,
+                       &hp));
+    *bytes = hp.total;
     return BEAM_MOE_OK;
   }
   // Sized for the largest split-K any device could pick (148 SMs bound it for

@@ -129,3 +129,32 @@ def test_trace_and_check_argument_errors():
     assert L.beam_moe_trace_create(0, ctypes.byref(h)) == INVALID
     assert L.beam_moe_trace_destroy(None) == INVALID
     assert L.beam_moe_check(None, 0, None, None) == INVALID
+
+
+def test_host_forward_workspace_and_argument_checks():
+    cfg = bm.beam_cfg()
+    H, C = 5120, bm.HOST_CHUNK
+    fwd = lambda T: bm.beam_moe_workspace_size(cfg, T, bm.OP_FORWARD)
+    host = lambda T, op=bm.OP_FORWARD_HOST: bm.beam_moe_workspace_size(cfg, T, op)
+    # one chunk: the forward's workspace plus one staging buffer each way
+    assert host(4096) >= fwd(4096) + 2 * 4096 * H * 2
+    # from two chunks on: one chunk's workspace plus two staging buffers each way,
+    # independent of T and far below the whole batch's forward workspace
+    assert host(7 * C) == host(2 * C) >= fwd(C) + 4 * C * H * 2
+    assert host(65536) == host(100000) >= fwd(2 * C) + 8 * C * H * 2  # bf16: 2C-token chunks
+    assert host(65536) < fwd(65536) // 2
+    assert host(65536, bm.OP_FORWARD_NVFP4_HOST) >= 4 * C * H * 2
+    L = bm.lib()
+    need = host(64)
+    a = 1 << 20  # fake but aligned addresses: never dereferenced on these paths
+    f = L.beam_moe_forward_host
+    assert f(ctypes.byref(cfg), 0, None, None, None, None, None, None, None, 0, None) == OK
+    assert f(ctypes.byref(cfg), 64, None, a, None, a, a, a, a, need, None) == INVALID
+    assert f(ctypes.byref(cfg), 64, a, a, None, a, a, None, a, need, None) == INVALID
+    assert f(ctypes.byref(cfg), 64, a, a, None, a, a, a, a + 8, need, None) == ALIGN
+    assert f(ctypes.byref(cfg), 64, a, a, None, a, a, a, a, need - 1, None) == WS_SMALL
+    assert f(ctypes.byref(cfg), 64, a, None, None, a, a, a, a, need, None) == INVALID
+    odd = bm.beam_cfg(H=320)  # hidden not a multiple of 256
+    ex = bm.BeamMoeNvfp4Experts(a, a, a, a, 1.0, 1.0, 1.0, 1.0)
+    assert L.beam_moe_forward_nvfp4_host(ctypes.byref(odd), 64, a, a, None, ctypes.byref(ex), a,
+                                         a, need, None) == UNSUPPORTED
