@@ -357,7 +357,8 @@ beam_moe_status forward_nvfp4_impl(const beam_moe_cfg* cfg, int64_t T, const uin
   BEAM_CUDA(rec.mark(4));
   BEAM_CUDA(beam::launch_gateup_nvfp4(*cfg, F, *ex, w, st));
   BEAM_CUDA(rec.mark(5));
-  BEAM_CUDA(beam::launch_down_nvfp4(*cfg, F, *ex, w, st));
+  BEAM_CUDA(F.pair_down ? beam::launch_down_nvfp4_pair(*cfg, F, *ex, w, st)
+                        : beam::launch_down_nvfp4(*cfg, F, *ex, w, st));
   BEAM_CUDA(rec.mark(6));
   BEAM_CUDA(beam::launch_combine(*cfg, L, out, w, st));
   BEAM_CUDA(rec.mark(7));

@@ -66,9 +66,11 @@ struct Fp4Layout {
   size_t xsf;     // uint8[rows * H/16] their scales (atom layout)
   size_t hq;      // uint8[rows * I/2] quantised h
   size_t hsf;     // uint8[rows * I/16]
+  int pair_down;  // 1: down GEMM on CTA pairs (nvfp4_2sm.cu)
 };
 Fp4Layout make_layout_nvfp4(const beam_moe_cfg& c, int64_t T, int sms);
 bool nvfp4_supported(const beam_moe_cfg& c);
+bool nvfp4_pair_supported(const beam_moe_cfg& c);
 
 // ---- launchers (each enqueues on `st`, returns cudaGetLastError()) --------
 // Router GEMM into the partial logits: the tensor-core kernel when
@@ -114,6 +116,8 @@ cudaError_t launch_permute_nvfp4(const beam_moe_cfg& c, const Fp4Layout& F, cons
                                  float gx, char* ws, cudaStream_t st);
 cudaError_t launch_gateup_nvfp4(const beam_moe_cfg& c, const Fp4Layout& F,
                                 const beam_moe_nvfp4_experts& w, char* ws, cudaStream_t st);
+cudaError_t launch_down_nvfp4_pair(const beam_moe_cfg& c, const Fp4Layout& F,
+                                   const beam_moe_nvfp4_experts& w, char* ws, cudaStream_t st);
 cudaError_t launch_down_nvfp4(const beam_moe_cfg& c, const Fp4Layout& F,
                               const beam_moe_nvfp4_experts& w, char* ws, cudaStream_t st);
 cudaError_t launch_quantize_rows(int64_t rows, int64_t K, const float* v, float g, uint8_t* codes,

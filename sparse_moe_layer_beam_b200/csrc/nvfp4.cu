@@ -580,6 +580,12 @@ Fp4Layout make_layout_nvfp4(const beam_moe_cfg& c, int64_t T, int sms) {
   Layout& L = F.base;
   L.bn = kBN;  // token tiles of 128 rows; expert segments padded to them
   L.pair_gateup = L.pair_down = 0;
+  // CTA pairs for the down GEMM once experts average 1024 rows or more. A
+  // pair tile of 256 weight rows x 256 tokens halves the operand bytes per
+  // FLOP, but its one 256-column accumulator leaves the MMAs idle while the
+  // epilogue drains it; measured, it wins only at the largest batches
+  // (T = 65536: 5.46 against 5.90 ms; T = 4096: 0.553 against 0.536 ms).
+  F.pair_down = ((double)T * c.top_k / c.n_experts >= 1024.0 && nvfp4_pair_supported(c)) ? 1 : 0;
   const int H = c.hidden, I = c.inter, E = c.n_experts;
   F.rows = ((L.A + kBN - 1) / kBN + E) * (int64_t)kBN;  // bound on the padded rows
   size_t o = L.route_end;

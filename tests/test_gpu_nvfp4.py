@@ -46,7 +46,7 @@ def test_device_nvfp4_weights_match_host():
     assert np.array_equal(ds, hs)
 
 
-@pytest.mark.parametrize("T", [64, 1, 129, 1024])
+@pytest.mark.parametrize("T", [64, 1, 129, 300, 1024, 4000, 4100])  # from 1024 rows/expert: pairs
 def test_nvfp4_forward_tiny(T):
     wl = TINY4.with_T(T)
     x, _, wr, b, r = _inputs.routed_inputs(wl)
