@@ -69,3 +69,27 @@ def test_nvfp4_decode_full_size():
     ref = _gpu.oracle_outputs_nvfp4(wl, x, tokens, r)
     err, rms = _gpu.max_rel_err(g["out"][tokens], ref)
     assert err <= _gpu.TOL, (err, rms)
+
+
+def _full_case(name, n_sample):
+    wl = synth.workload(name)
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    g = _gpu.forward_nvfp4(wl, x, bias=b)
+    assert g["flags"] == 0
+    _gpu.check_routes(g, r, wl.E)
+    tokens = synth.sample_tokens(wl.T, n_sample)
+    ref = _gpu.oracle_outputs_nvfp4(wl, x, tokens, r)
+    err, rms = _gpu.max_rel_err(g["out"][tokens], ref)
+    assert err <= _gpu.TOL, (err, rms)
+
+
+def test_nvfp4_prefill_full_size():
+    _full_case("prefill", 8)
+
+
+def test_nvfp4_skewed_full_size():  # router bias on the logits of 16 hot experts
+    _full_case("skewed", 8)
+
+
+def test_nvfp4_long_full_size():  # 2048 rows per expert: the down GEMM runs on CTA pairs
+    _full_case("long", 8)
