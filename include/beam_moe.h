@@ -277,6 +277,80 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_traced(const beam_moe_cfg* cfg, in
                                         void* stream, beam_moe_trace* trace);
 
 /*
+ * Expert parallelism. `world` ranks (one per GPU) each hold E / world
+ * consecutive experts and route their own tokens; the block's arithmetic is
+ * beam_moe_forward's, split over the ranks (the DEP / all-to-all layout the
+ * vLLM recipe and DeepEP use for Beam, "Welcome Beam" and the vLLM recipe).
+ * A rank calls, in order:
+ *   1 beam_moe_ep_route     routes its T tokens, writes counts [E] (device)
+ *   -                       the caller all-gathers counts into counts_all
+ *                           [world][E] on the host
+ *   2 beam_moe_ep_plan      (host) where this rank's rows land in every
+ *                           owner's receive buffer, and what it receives
+ *   3 beam_moe_ep_dispatch  writes its token rows and their return
+ *                           addresses into the owners' workspaces
+ *   -                       barrier: every rank's dispatch has completed
+ *   4 beam_moe_ep_experts   grouped GEMMs over the received rows, each y row
+ *                           written back into its source rank's workspace
+ *   -                       barrier: every rank's experts call has completed
+ *   5 beam_moe_ep_combine   out[t] = sum_k w[t][k] y[t][k], fixed k order
+ * No kernel waits for another rank: the caller orders the phases (an NCCL
+ * all-gather and barriers, or stream order when all ranks share one GPU).
+ * peer_ws[r] is rank r's workspace as a pointer this rank's GPU can store
+ * to (NVLink peer memory; the same allocation when r == rank). Every rank's
+ * workspace has the same size and layout (same cfg, world, t_max,
+ * recv_cap); routes, returned rows and scratch stay in it from route to
+ * combine. Rank r owns experts [r E / world, (r + 1) E / world).
+ */
+typedef struct beam_moe_ep_cfg {
+  int32_t world;    /* ranks, 1..8, dividing n_experts                        */
+  int32_t rank;     /* this rank, 0..world-1                                  */
+  int64_t t_max;    /* most tokens a rank routes in one call                  */
+  int64_t recv_cap; /* rows a rank's receive buffer holds (beam_moe_ep_plan
+                       fails when any rank would receive more)                 */
+} beam_moe_ep_cfg;
+BEAM_MOE_API beam_moe_status beam_moe_ep_workspace_size(const beam_moe_cfg* cfg,
+                                                        const beam_moe_ep_cfg* ep,
+                                                        size_t* bytes);
+/* counts [E] int32, device (out): this rank's tokens routed to each expert. */
+BEAM_MOE_API beam_moe_status beam_moe_ep_route(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep,
+                                               int64_t T, const uint16_t* x,
+                                               const float* w_router, const float* bias,
+                                               int32_t* counts, void* ws, size_t ws_bytes,
+                                               void* stream);
+/* Host only. counts_all [world][E] int32 (host): every rank's counts.
+ * send_base [E] int32 (host, out): first row, in the owner's receive buffer,
+ * of this rank's rows for each expert (its rows for an expert are in token
+ * order; sources follow one another in rank order). recv_counts [E/world]
+ * int32 (host, out): rows this rank receives per local expert; *recv_rows
+ * their sum. Fails with BEAM_MOE_ERR_WORKSPACE_TOO_SMALL if any rank would
+ * receive more than recv_cap rows (every rank reaches the same verdict). */
+BEAM_MOE_API beam_moe_status beam_moe_ep_plan(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep,
+                                              const int32_t* counts_all, int32_t* send_base,
+                                              int32_t* recv_counts, int64_t* recv_rows);
+/* x [T][H] bf16, device: the tokens routed by beam_moe_ep_route (same T).
+ * send_base [E] int32, device: beam_moe_ep_plan's, copied to the device.
+ * peer_ws [world] (host array of device pointers). */
+BEAM_MOE_API beam_moe_status beam_moe_ep_dispatch(const beam_moe_cfg* cfg,
+                                                  const beam_moe_ep_cfg* ep, int64_t T,
+                                                  const uint16_t* x, const int32_t* send_base,
+                                                  void* const* peer_ws, void* ws,
+                                                  size_t ws_bytes, void* stream);
+/* recv_counts [E/world] int32 (host): beam_moe_ep_plan's. w13, w2: this
+ * rank's experts only ([E/world][2I][H], [E/world][H][I] bf16, device). */
+BEAM_MOE_API beam_moe_status beam_moe_ep_experts(const beam_moe_cfg* cfg,
+                                                 const beam_moe_ep_cfg* ep,
+                                                 const int32_t* recv_counts,
+                                                 const uint16_t* w13, const uint16_t* w2,
+                                                 void* const* peer_ws, void* ws,
+                                                 size_t ws_bytes, void* stream);
+/* out [T][H] bf16, device (same T as the route call). */
+BEAM_MOE_API beam_moe_status beam_moe_ep_combine(const beam_moe_cfg* cfg,
+                                                 const beam_moe_ep_cfg* ep, int64_t T,
+                                                 uint16_t* out, void* ws, size_t ws_bytes,
+                                                 void* stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the device status word in the
  * workspace. *device_flags (may be NULL) receives the raw bits: 0x1 producer,
  * 0x2 MMA issuer, 0x4 epilogue gave up a bounded wait; 0x100 an expert id

@@ -19,7 +19,9 @@ __all__ = ["BeamMoeCfg", "BeamMoeError", "Trace", "OP_ROUTE", "OP_FORWARD", "N_S
            "beam_moe_route_noalloc", "BeamMoeNvfp4Experts", "OP_FORWARD_NVFP4", "nvfp4_experts",
            "beam_moe_forward_nvfp4", "beam_moe_nvfp4_quantize", "OP_FORWARD_HOST",
            "OP_FORWARD_NVFP4_HOST", "HOST_CHUNK", "beam_moe_forward_host",
-           "beam_moe_forward_nvfp4_host",
+           "beam_moe_forward_nvfp4_host", "BeamMoeEpCfg", "ep_cfg", "beam_moe_ep_workspace_size",
+           "beam_moe_ep_route", "beam_moe_ep_plan", "beam_moe_ep_dispatch", "beam_moe_ep_experts",
+           "beam_moe_ep_combine",
            "beam_moe_forward", "beam_moe_forward_routed", "beam_moe_forward_traced",
            "beam_moe_check"]
 
@@ -53,6 +55,12 @@ class BeamMoeNvfp4Experts(ctypes.Structure):
                 ("x_scale", ctypes.c_float), ("h_scale", ctypes.c_float)]
 
 
+class BeamMoeEpCfg(ctypes.Structure):
+    """Expert parallelism: ranks, this rank, most tokens per rank, receive rows."""
+    _fields_ = [("world", ctypes.c_int32), ("rank", ctypes.c_int32), ("t_max", ctypes.c_int64),
+                ("recv_cap", ctypes.c_int64)]
+
+
 class BeamMoeError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
@@ -62,6 +70,8 @@ class BeamMoeError(RuntimeError):
 _lib = None
 _P = ctypes.c_void_p
 _CFG = ctypes.POINTER(BeamMoeCfg)
+_EP = ctypes.POINTER(BeamMoeEpCfg)
+_PP = ctypes.POINTER(ctypes.c_void_p)
 _SIGS = {
     "beam_moe_workspace_size": [_CFG, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)],
     "beam_moe_route": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
@@ -84,6 +94,12 @@ _SIGS = {
                                     ctypes.POINTER(BeamMoeNvfp4Experts), _P, _P, ctypes.c_size_t,
                                     _P],
     "beam_moe_nvfp4_quantize": [ctypes.c_int64, ctypes.c_int64, _P, ctypes.c_float, _P, _P, _P],
+    "beam_moe_ep_workspace_size": [_CFG, _EP, ctypes.POINTER(ctypes.c_size_t)],
+    "beam_moe_ep_route": [_CFG, _EP, ctypes.c_int64, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "beam_moe_ep_plan": [_CFG, _EP, _P, _P, _P, ctypes.POINTER(ctypes.c_int64)],
+    "beam_moe_ep_dispatch": [_CFG, _EP, ctypes.c_int64, _P, _P, _PP, _P, ctypes.c_size_t, _P],
+    "beam_moe_ep_experts": [_CFG, _EP, _P, _P, _P, _PP, _P, ctypes.c_size_t, _P],
+    "beam_moe_ep_combine": [_CFG, _EP, ctypes.c_int64, _P, _P, ctypes.c_size_t, _P],
     "beam_moe_trace_create": [ctypes.c_int32, ctypes.POINTER(_P)],
     "beam_moe_trace_destroy": [_P],
     "beam_moe_trace_reset": [_P],
@@ -269,3 +285,69 @@ class Trace:
             self.close()
         except Exception:
             pass
+
+
+# ------------------------------------------------------------ expert parallelism
+
+def ep_cfg(world, rank, t_max, recv_cap):
+    return BeamMoeEpCfg(world, rank, t_max, recv_cap)
+
+
+def _addr(v):
+    return v if isinstance(v, int) or v is None else v.data_ptr()
+
+
+def _peers(peer_ws):
+    return (ctypes.c_void_p * len(peer_ws))(*[_addr(p) for p in peer_ws])
+
+
+def beam_moe_ep_workspace_size(cfg, ep):
+    n = ctypes.c_size_t(0)
+    _check(lib().beam_moe_ep_workspace_size(ctypes.byref(cfg), ctypes.byref(ep), ctypes.byref(n)),
+           "beam_moe_ep_workspace_size")
+    return n.value
+
+
+def beam_moe_ep_route(cfg, ep, x, w_router, bias, counts, ws, stream=None):
+    _check(lib().beam_moe_ep_route(ctypes.byref(cfg), ctypes.byref(ep), x.shape[0], _ptr(x),
+                                   _ptr(w_router), _ptr(bias), _ptr(counts), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)),
+           "beam_moe_ep_route")
+
+
+def beam_moe_ep_plan(cfg, ep, counts_all):
+    """counts_all: int32 array [world][E] (host). Returns (send_base [E],
+    recv_counts [E/world], recv_rows)."""
+    import numpy as np
+    counts_all = np.ascontiguousarray(counts_all, dtype=np.int32)
+    send_base = np.zeros(cfg.n_experts, dtype=np.int32)
+    recv_counts = np.zeros(cfg.n_experts // ep.world, dtype=np.int32)
+    rows = ctypes.c_int64(0)
+    _check(lib().beam_moe_ep_plan(ctypes.byref(cfg), ctypes.byref(ep), counts_all.ctypes.data,
+                                  send_base.ctypes.data, recv_counts.ctypes.data,
+                                  ctypes.byref(rows)), "beam_moe_ep_plan")
+    return send_base, recv_counts, rows.value
+
+
+def beam_moe_ep_dispatch(cfg, ep, x, send_base, peer_ws, ws, stream=None):
+    _check(lib().beam_moe_ep_dispatch(ctypes.byref(cfg), ctypes.byref(ep), x.shape[0], _ptr(x),
+                                      _ptr(send_base), _peers(peer_ws), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)),
+           "beam_moe_ep_dispatch")
+
+
+def beam_moe_ep_experts(cfg, ep, recv_counts, w13, w2, peer_ws, ws, stream=None):
+    """recv_counts: int32 array [E/world] (host); w13, w2: this rank's experts
+    (tensors or device addresses)."""
+    import numpy as np
+    rc = np.ascontiguousarray(recv_counts, dtype=np.int32)
+    _check(lib().beam_moe_ep_experts(ctypes.byref(cfg), ctypes.byref(ep), rc.ctypes.data,
+                                     _addr(w13), _addr(w2), _peers(peer_ws), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)),
+           "beam_moe_ep_experts")
+
+
+def beam_moe_ep_combine(cfg, ep, T, out, ws, stream=None):
+    _check(lib().beam_moe_ep_combine(ctypes.byref(cfg), ctypes.byref(ep), T, _ptr(out), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)),
+           "beam_moe_ep_combine")

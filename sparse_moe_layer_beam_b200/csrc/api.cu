@@ -692,6 +692,238 @@ beam_moe_status beam_moe_trace_read(beam_moe_trace* t, float* ms, int32_t* n_cal
   return BEAM_MOE_OK;
 }
 
+// ------------------------------------------------------ expert parallelism
+}  // extern "C"
+
+namespace {
+
+beam_moe_status ep_checks(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep) {
+  BEAM_TRY(check_cfg(cfg));
+  if (!ep) return BEAM_MOE_ERR_INVALID_ARG;
+  if (ep->world < 1 || ep->world > 8 || ep->rank < 0 || ep->rank >= ep->world ||
+      ep->t_max < 0 || ep->recv_cap < 0)
+    return BEAM_MOE_ERR_INVALID_ARG;
+  if (cfg->n_experts % ep->world != 0) return BEAM_MOE_ERR_UNSUPPORTED_SHAPE;
+  // return addresses hold the source rank above 27 bits of token slot
+  if (ep->t_max * cfg->top_k >= ((int64_t)1 << 27) || ep->recv_cap >= ((int64_t)1 << 31))
+    return BEAM_MOE_ERR_UNSUPPORTED_SHAPE;
+  BEAM_TRY(check_T(cfg, ep->t_max));
+  return BEAM_MOE_OK;
+}
+
+// The routing layout of T tokens, moved to start at `base` of the workspace;
+// its status word is the workspace's first (shared with the expert stage).
+Layout ep_routing(const beam_moe_cfg& c, int64_t T, int sms, size_t base) {
+  Layout L = beam::make_layout(c, T, sms);
+  size_t* f[] = {&L.counts, &L.offsets, &L.nb_off, &L.nb2_off, &L.ids, &L.w, &L.pos,
+                 &L.chunk_cnt, &L.chunk_mask, &L.logits, &L.w3, &L.route_end, &L.xp, &L.h,
+                 &L.total};
+  for (size_t* v : f) *v += base;
+  L.status = 0;
+  return L;
+}
+
+// Routing scratch for any T <= t_max. Its size is not monotone in T (the
+// router's split over H depends on T), so take the maximum: every T up to
+// 4096, then the last T of every 128-token block (both routers' token tiles
+// are whole 128-token blocks there, so within one block the split is fixed
+// and the size grows with T).
+size_t ep_route_bytes(const beam_moe_cfg& c, int64_t t_max) {
+  size_t best = 0;
+  for (int64_t t = 1; t <= t_max; t = (t < 4096 ? t + 1 : (t + 128) / 128 * 128)) {
+    const Layout L = beam::make_layout(c, t, 1024);
+    if (L.route_end > best) best = L.route_end;
+    if (t >= 4096 && t + 128 > t_max && t != t_max) {
+      const Layout M = beam::make_layout(c, t_max, 1024);
+      if (M.route_end > best) best = M.route_end;
+      break;
+    }
+  }
+  return best;
+}
+
+beam_moe_status ep_ws_checks(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep, void* ws,
+                             size_t ws_bytes) {
+  if (!ws) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return BEAM_MOE_ERR_ALIGNMENT;
+  size_t need = 0;
+  BEAM_TRY(beam_moe_ep_workspace_size(cfg, ep, &need));
+  if (ws_bytes < need) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+  return BEAM_MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+beam_moe_status beam_moe_ep_workspace_size(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep,
+                                           size_t* bytes) {
+  BEAM_TRY(ep_checks(cfg, ep));
+  if (!bytes) return BEAM_MOE_ERR_INVALID_ARG;
+  const beam::EpLayout P = beam::make_ep_layout(*cfg, *ep);
+  *bytes = P.route + ep_route_bytes(*cfg, ep->t_max);
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_ep_route(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep, int64_t T,
+                                  const uint16_t* x, const float* w_router, const float* bias,
+                                  int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  BEAM_TRY(ep_checks(cfg, ep));
+  if (T < 0 || T > ep->t_max) return BEAM_MOE_ERR_INVALID_ARG;
+  BEAM_TRY(ep_ws_checks(cfg, ep, ws, ws_bytes));
+  BEAM_TRY(check_ptrs({counts}, {}));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  BEAM_CUDA(cudaMemsetAsync(w, 0, 256, st));
+  if (T == 0) {
+    BEAM_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, st));
+    return BEAM_MOE_OK;
+  }
+  BEAM_TRY(check_ptrs({x, w_router}, {bias}));
+  const beam::EpLayout P = beam::make_ep_layout(*cfg, *ep);
+  const Layout L = ep_routing(*cfg, T, beam::device_sm_count(), P.route);
+  BEAM_CUDA(beam::launch_router_logits(*cfg, L, x, w_router, w, st));
+  BEAM_CUDA(beam::launch_router_topk(*cfg, L, bias, w, st));
+  BEAM_CUDA(beam::launch_scan(*cfg, L, w, counts, st));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_ep_plan(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep,
+                                 const int32_t* counts_all, int32_t* send_base,
+                                 int32_t* recv_counts, int64_t* recv_rows) {
+  BEAM_TRY(ep_checks(cfg, ep));
+  if (!counts_all || !send_base || !recv_counts || !recv_rows) return BEAM_MOE_ERR_INVALID_ARG;
+  const int E = cfg->n_experts, W = ep->world, El = E / W;
+  for (int s = 0; s < W; ++s) {
+    int64_t sum = 0;
+    for (int e = 0; e < E; ++e) {
+      const int32_t v = counts_all[(size_t)s * E + e];
+      if (v < 0) return BEAM_MOE_ERR_INVALID_ARG;
+      sum += v;
+    }
+    if (sum > ep->t_max * cfg->top_k) return BEAM_MOE_ERR_INVALID_ARG;
+  }
+  // owner o's receive buffer: local experts in order, each expert's rows
+  // from source 0, then source 1, ...
+  for (int o = 0; o < W; ++o) {
+    int64_t row = 0;
+    for (int j = 0; j < El; ++j) {
+      const int e = o * El + j;
+      int64_t got = 0;
+      for (int s = 0; s < W; ++s) {
+        if (s == ep->rank) send_base[e] = (int32_t)(row + got);
+        got += counts_all[(size_t)s * E + e];
+      }
+      if (o == ep->rank) recv_counts[j] = (int32_t)got;
+      row += got;
+    }
+    if (row > ep->recv_cap) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (o == ep->rank) *recv_rows = row;
+  }
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_ep_dispatch(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep,
+                                     int64_t T, const uint16_t* x, const int32_t* send_base,
+                                     void* const* peer_ws, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  BEAM_TRY(ep_checks(cfg, ep));
+  if (T < 0 || T > ep->t_max) return BEAM_MOE_ERR_INVALID_ARG;
+  BEAM_TRY(ep_ws_checks(cfg, ep, ws, ws_bytes));
+  if (T == 0) return BEAM_MOE_OK;
+  BEAM_TRY(check_ptrs({x, send_base}, {}));
+  if (!peer_ws) return BEAM_MOE_ERR_INVALID_ARG;
+  for (int r = 0; r < ep->world; ++r)
+    if (!peer_ws[r] || !aligned16(peer_ws[r])) return BEAM_MOE_ERR_INVALID_ARG;
+  if (peer_ws[ep->rank] != ws) return BEAM_MOE_ERR_INVALID_ARG;
+  const beam::EpLayout P = beam::make_ep_layout(*cfg, *ep);
+  const Layout L = ep_routing(*cfg, T, beam::device_sm_count(), P.route);
+  BEAM_CUDA(beam::launch_ep_dispatch(*cfg, *ep, P, L, x, send_base, peer_ws,
+                                     static_cast<char*>(ws), reinterpret_cast<cudaStream_t>(stream)));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_ep_experts(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep,
+                                    const int32_t* recv_counts, const uint16_t* w13,
+                                    const uint16_t* w2, void* const* peer_ws, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  BEAM_TRY(ep_checks(cfg, ep));
+  BEAM_TRY(ep_ws_checks(cfg, ep, ws, ws_bytes));
+  if (!recv_counts || !peer_ws) return BEAM_MOE_ERR_INVALID_ARG;
+  const int El = cfg->n_experts / ep->world;
+  std::vector<int32_t> counts(El), offsets(El + 1), nb_off(El + 1);
+  int64_t rows = 0;
+  for (int j = 0; j < El; ++j) {
+    if (recv_counts[j] < 0) return BEAM_MOE_ERR_INVALID_ARG;
+    counts[j] = recv_counts[j];
+    offsets[j] = (int32_t)rows;
+    rows += recv_counts[j];
+  }
+  offsets[El] = (int32_t)rows;
+  if (rows > ep->recv_cap) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (rows == 0) return BEAM_MOE_OK;
+  BEAM_TRY(check_ptrs({w13, w2}, {}));
+  for (int r = 0; r < ep->world; ++r)
+    if (!peer_ws[r] || !aligned16(peer_ws[r])) return BEAM_MOE_ERR_INVALID_ARG;
+  if (peer_ws[ep->rank] != ws) return BEAM_MOE_ERR_INVALID_ARG;
+  // the received rows as the grouped GEMMs' permuted rows, over the local
+  // experts; token tile and CTA pairs chosen as for a forward
+  beam_moe_cfg lc = *cfg;
+  lc.n_experts = El;
+  const beam::EpLayout P = beam::make_ep_layout(*cfg, *ep);
+  Layout L;
+  memset(&L, 0, sizeof(L));
+  L.A = rows;
+  L.T = rows;
+  L.bn = beam::pick_bn(rows, 1, El);
+  const double mean = (double)rows / El;
+  const bool pair_ok = L.bn == 256 && beam::pair_gemm_supported(lc);
+  L.pair_gateup = L.pair_down = (pair_ok && mean >= 64.0) ? 1 : 0;
+  L.status = P.status;
+  L.counts = P.counts;
+  L.offsets = P.offsets;
+  L.nb_off = P.nb_off;
+  L.nb2_off = P.nb2_off;
+  L.xp = P.recv;
+  L.h = P.h;
+  int32_t acc = 0;
+  for (int j = 0; j < El; ++j) {
+    nb_off[j] = acc;
+    acc += (counts[j] + L.bn - 1) / L.bn;
+  }
+  nb_off[El] = acc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  BEAM_CUDA(cudaMemcpyAsync(w + P.counts, counts.data(), 4 * El, cudaMemcpyHostToDevice, st));
+  BEAM_CUDA(cudaMemcpyAsync(w + P.offsets, offsets.data(), 4 * (El + 1), cudaMemcpyHostToDevice, st));
+  BEAM_CUDA(cudaMemcpyAsync(w + P.nb_off, nb_off.data(), 4 * (El + 1), cudaMemcpyHostToDevice, st));
+  BEAM_CUDA(cudaStreamSynchronize(st));  // the host arrays are this call's
+  BEAM_CUDA(L.pair_gateup ? beam::launch_gateup_pair(lc, L, w13, w, st)
+                          : beam::launch_gateup(lc, L, w13, w, st));
+  BEAM_CUDA(L.pair_down ? beam::launch_down_pair(lc, L, w2, w, st)
+                        : beam::launch_down(lc, L, w2, w, st));
+  BEAM_CUDA(beam::launch_ep_return(*cfg, *ep, P, rows, peer_ws, w, st));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_ep_combine(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep,
+                                    int64_t T, uint16_t* out, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  BEAM_TRY(ep_checks(cfg, ep));
+  if (T < 0 || T > ep->t_max) return BEAM_MOE_ERR_INVALID_ARG;
+  BEAM_TRY(ep_ws_checks(cfg, ep, ws, ws_bytes));
+  if (T == 0) return BEAM_MOE_OK;
+  BEAM_TRY(check_ptrs({out}, {}));
+  const beam::EpLayout P = beam::make_ep_layout(*cfg, *ep);
+  const Layout L = ep_routing(*cfg, T, beam::device_sm_count(), P.route);
+  char* w = static_cast<char*>(ws);
+  BEAM_CUDA(beam::launch_combine_from(*cfg, T, reinterpret_cast<const float*>(w + P.yret),
+                                      reinterpret_cast<const int32_t*>(w + L.pos),
+                                      reinterpret_cast<const float*>(w + L.w), out,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+  return BEAM_MOE_OK;
+}
+
 beam_moe_status beam_moe_check(void* ws, size_t ws_bytes, void* stream, uint32_t* device_flags) {
   if (!ws || ws_bytes < 256) return BEAM_MOE_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -214,6 +214,14 @@ cudaError_t launch_combine(const beam_moe_cfg& c, const Layout& L, uint16_t* out
   return cudaGetLastError();
 }
 
+cudaError_t launch_combine_from(const beam_moe_cfg& c, int64_t T, const float* y,
+                                const int32_t* pos, const float* w, uint16_t* out,
+                                cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  combine_kernel<<<(unsigned)T, 128, 0, st>>>(y, c.hidden, c.top_k, pos, w, out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_copy_routes(const beam_moe_cfg& c, const Layout& L, int32_t* ids_out,
                                float* w_out, char* ws, cudaStream_t st) {
   const size_t n = (size_t)L.A;

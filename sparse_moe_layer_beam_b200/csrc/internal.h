@@ -72,7 +72,26 @@ Fp4Layout make_layout_nvfp4(const beam_moe_cfg& c, int64_t T, int sms);
 bool nvfp4_supported(const beam_moe_cfg& c);
 bool nvfp4_pair_supported(const beam_moe_cfg& c);
 
+// Expert parallelism: byte offsets inside every rank's workspace (identical
+// across ranks, so that peers can store into it). `route` is where the
+// routing layout of the rank's own tokens starts.
+struct EpLayout {
+  size_t status, recv, src, yret, h, counts, offsets, nb_off, nb2_off, route;
+};
+EpLayout make_ep_layout(const beam_moe_cfg& c, const beam_moe_ep_cfg& g);
+
 // ---- launchers (each enqueues on `st`, returns cudaGetLastError()) --------
+// EP: token rows and return addresses to the owners; y rows back to sources.
+// L is the routing layout with offsets relative to ws.
+cudaError_t launch_ep_dispatch(const beam_moe_cfg& c, const beam_moe_ep_cfg& g,
+                               const EpLayout& P, const Layout& L, const uint16_t* x,
+                               const int32_t* send_base, void* const* peer_ws, char* ws,
+                               cudaStream_t st);
+cudaError_t launch_ep_return(const beam_moe_cfg& c, const beam_moe_ep_cfg& g, const EpLayout& P,
+                             int64_t rows, void* const* peer_ws, char* ws, cudaStream_t st);
+cudaError_t launch_combine_from(const beam_moe_cfg& c, int64_t T, const float* y,
+                                const int32_t* pos, const float* w, uint16_t* out,
+                                cudaStream_t st);
 // Router GEMM into the partial logits: the tensor-core kernel when
 // L.router_tc, else the CUDA-core kernel. Either clears the dispatch bits.
 cudaError_t launch_router_logits(const beam_moe_cfg& c, const Layout& L, const uint16_t* x,

@@ -1,0 +1,79 @@
+"""Expert parallelism, with `world` ranks emulated on one GPU: every rank has
+its own workspace, peer pointers are the other ranks' workspaces, and the
+phases run rank after rank (a device synchronisation stands for each barrier).
+The kernels are the ones a multi-GPU run uses; only the peer stores stay on
+one device. Each rank's output must match the oracle and a single-GPU forward
+of the same tokens."""
+import numpy as np
+import pytest
+import torch
+
+import sparse_moe_layer_beam_b200 as bm
+import synth
+from tests import _gpu, _inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def ep_forward(wl, xs, world, bias=None):
+    cfg = _gpu.cfg_of(wl)
+    w13, w2, wr = _gpu.device_weights(wl)
+    El, H = wl.E // world, wl.H
+    Ts = [x.shape[0] for x in xs]
+    cap = sum(Ts) * min(wl.K, El)
+    eps = [bm.ep_cfg(world, r, max(Ts), cap) for r in range(world)]
+    wss = [torch.empty(bm.beam_moe_ep_workspace_size(cfg, ep), dtype=torch.uint8, device="cuda")
+           for ep in eps]
+    peers = [ws.data_ptr() for ws in wss]
+    xd = [_gpu.to_dev_bits(x) if x.shape[0] else torch.empty((0, H), dtype=torch.int16,
+                                                              device="cuda") for x in xs]
+    b = None if bias is None else torch.from_numpy(np.asarray(bias, np.float32)).cuda()
+    counts = [torch.empty(wl.E, dtype=torch.int32, device="cuda") for _ in range(world)]
+    for r in range(world):
+        bm.beam_moe_ep_route(cfg, eps[r], xd[r], wr, b, counts[r], wss[r])
+    counts_all = np.stack([c.cpu().numpy() for c in counts])  # the all-gather
+    plans = [bm.beam_moe_ep_plan(cfg, eps[r], counts_all) for r in range(world)]
+    for r in range(world):
+        bm.beam_moe_ep_dispatch(cfg, eps[r], xd[r], torch.from_numpy(plans[r][0]).cuda(), peers,
+                                wss[r])
+    torch.cuda.synchronize()  # barrier: every dispatch has landed
+    w13_bytes, w2_bytes = 2 * wl.I * wl.H * 2, wl.H * wl.I * 2  # one expert's weights
+    for r in range(world):
+        bm.beam_moe_ep_experts(cfg, eps[r], plans[r][1], w13.data_ptr() + r * El * w13_bytes,
+                               w2.data_ptr() + r * El * w2_bytes, peers, wss[r])
+    torch.cuda.synchronize()  # barrier: every y row is back at its source
+    outs = []
+    for r in range(world):
+        out = torch.empty((Ts[r], H), dtype=torch.int16, device="cuda")
+        bm.beam_moe_ep_combine(cfg, eps[r], Ts[r], out, wss[r])
+        outs.append(_gpu.bits_of(out))
+    for ws in wss:
+        assert bm.beam_moe_check(ws) == 0
+    return outs, counts_all, plans
+
+
+def _check(wl, world, Ts, n_sample=None):
+    T = sum(Ts)
+    x, _, wr, b, r = _inputs.routed_inputs(wl.with_T(T))
+    xs = np.split(x, np.cumsum(Ts)[:-1])
+    outs, counts_all, plans = ep_forward(wl, xs, world, b)
+    assert sum(p[2] for p in plans) == T * wl.K  # every assignment received once
+    got = np.concatenate(outs)
+    tokens = np.arange(T) if n_sample is None else synth.sample_tokens(T, n_sample)
+    ref = _gpu.oracle_outputs(wl.with_T(T), x, tokens, r)
+    err, rms = _gpu.max_rel_err(got[tokens], ref)
+    assert err <= _gpu.TOL, (err, rms)
+    for xr, o in zip(xs, outs):  # the same tokens through one GPU's forward
+        if xr.shape[0]:
+            single = _gpu.forward(wl.with_T(xr.shape[0]), xr, bias=b)["out"]
+            err, rms = _gpu.max_rel_err(o, synth.bf16_to_f32(single).astype(np.float64))
+            assert err <= _gpu.TOL, (err, rms)
+
+
+@pytest.mark.parametrize("world,Ts", [(1, [77]), (2, [100, 37]), (4, [64, 1, 129, 0])])
+def test_ep_tiny(world, Ts):
+    _check(synth.workload("tiny"), world, Ts)
+
+
+def test_ep_decode_full_size_eight_ranks():  # 32 experts per rank, 64 tokens each
+    _check(synth.workload("decode"), 8, [64] * 8, n_sample=12)

@@ -58,3 +58,60 @@ def test_reference_arm_prints_on_rank0_only():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _ep_worker(rank, world, port, out):
+    """Expert-parallel exchange logic: counts all-gathered over the process
+    group, every rank's plan, and a cross-check that each owner's receive
+    layout is exactly what the senders will write (world size 2, gloo)."""
+    import torch
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import sparse_moe_layer_beam_b200 as bm
+
+    cfg = bm.beam_cfg()
+    E, El, K = cfg.n_experts, cfg.n_experts // world, cfg.top_k
+    t_local = 50 + 30 * rank
+    rng = np.random.default_rng(100 + rank)
+    ids = np.stack([rng.choice(E, size=K, replace=False) for _ in range(t_local)])
+    counts = np.bincount(ids.ravel(), minlength=E).astype(np.int32)
+    gathered = [torch.zeros(E, dtype=torch.int32) for _ in range(world)]
+    dist.all_gather(gathered, torch.from_numpy(counts))
+    counts_all = torch.stack(gathered).numpy()
+    ep = bm.ep_cfg(world, rank, 80, world * 80 * K)
+    send_base, recv_counts, recv_rows = bm.beam_moe_ep_plan(cfg, ep, counts_all)
+    sends = [torch.zeros(E, dtype=torch.int32) for _ in range(world)]
+    dist.all_gather(sends, torch.from_numpy(send_base))
+    sends = torch.stack(sends).numpy()
+    # this rank as owner: every source's rows for each local expert are one
+    # contiguous run, in expert then source order, tiling [0, recv_rows)
+    row, ok = 0, True
+    for j in range(El):
+        e = rank * El + j
+        for s in range(world):
+            ok &= bool(sends[s, e] == row)
+            row += counts_all[s, e]
+    ok &= row == recv_rows == int(recv_counts.sum())
+    out.put((rank, ok, int(recv_rows), int(counts_all.sum())))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_expert_parallel_plan_over_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 31500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_ep_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, ok0, rows0, tot0), (r1, ok1, rows1, tot1) = res
+    assert ok0 and ok1
+    assert tot0 == tot1 == (50 + 80) * 8        # every assignment of both ranks
+    assert rows0 + rows1 == tot0                 # received exactly once, by its owner
