@@ -354,10 +354,22 @@ BEAM_MOE_API beam_moe_status beam_moe_ep_combine(const beam_moe_cfg* cfg,
  * Synchronizes `stream`, then reads and clears the device status word in the
  * workspace. *device_flags (may be NULL) receives the raw bits: 0x1 producer,
  * 0x2 MMA issuer, 0x4 epilogue gave up a bounded wait; 0x100 an expert id
- * outside [0, E) reached the dispatch. Returns BEAM_MOE_ERR_DEVICE_TIMEOUT
+ * outside [0, E) reached the dispatch; 0x200 beam_moe_selftest_wait's wait ran
+ * out. Returns BEAM_MOE_ERR_DEVICE_TIMEOUT
  * if any bit was set, BEAM_MOE_ERR_CUDA if the stream reports an error.
  */
 BEAM_MOE_API beam_moe_status beam_moe_check(void* ws, size_t ws_bytes, void* stream, uint32_t* device_flags);
+
+/*
+ * Device self-check of the failure path: one thread waits on an mbarrier that
+ * nothing completes; after limit_ms (1..1000) the wait gives up, sets status
+ * bit 0x200 in the workspace's status word and the kernel returns, exactly as
+ * a tensor-core kernel of this library does when one of its bounded waits
+ * runs out. beam_moe_check then reports BEAM_MOE_ERR_DEVICE_TIMEOUT with that
+ * bit, and the context stays usable. ws: at least 256 bytes, device.
+ */
+BEAM_MOE_API beam_moe_status beam_moe_selftest_wait(void* ws, size_t ws_bytes, int32_t limit_ms,
+                                                    void* stream);
 
 /* Static description of a status code. */
 BEAM_MOE_API const char* beam_moe_status_string(beam_moe_status status);

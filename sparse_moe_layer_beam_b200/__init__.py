@@ -21,7 +21,7 @@ __all__ = ["BeamMoeCfg", "BeamMoeError", "Trace", "OP_ROUTE", "OP_FORWARD", "N_S
            "OP_FORWARD_NVFP4_HOST", "HOST_CHUNK", "beam_moe_forward_host",
            "beam_moe_forward_nvfp4_host", "BeamMoeEpCfg", "ep_cfg", "beam_moe_ep_workspace_size",
            "beam_moe_ep_route", "beam_moe_ep_plan", "beam_moe_ep_dispatch", "beam_moe_ep_experts",
-           "beam_moe_ep_combine",
+           "beam_moe_ep_combine", "beam_moe_selftest_wait",
            "beam_moe_forward", "beam_moe_forward_routed", "beam_moe_forward_traced",
            "beam_moe_check"]
 
@@ -105,6 +105,7 @@ _SIGS = {
     "beam_moe_trace_reset": [_P],
     "beam_moe_trace_read": [_P, _P, ctypes.POINTER(ctypes.c_int32)],
     "beam_moe_check": [_P, ctypes.c_size_t, _P, ctypes.POINTER(ctypes.c_uint32)],
+    "beam_moe_selftest_wait": [_P, ctypes.c_size_t, ctypes.c_int32, _P],
     "beam_moe_status_string": [ctypes.c_int],
 }
 
@@ -254,6 +255,12 @@ def beam_moe_check(ws, stream=None):
     if st not in (0, 6):
         raise BeamMoeError(st, "beam_moe_check")
     return flags.value
+
+
+def beam_moe_selftest_wait(ws, limit_ms, stream=None):
+    """Runs the device self-check of a bounded wait that runs out."""
+    _check(lib().beam_moe_selftest_wait(_ptr(ws), ws.numel() * ws.element_size(), limit_ms,
+                                        _stream(stream)), "beam_moe_selftest_wait")
 
 
 class Trace:

@@ -937,6 +937,15 @@ beam_moe_status beam_moe_check(void* ws, size_t ws_bytes, void* stream, uint32_t
   return flags ? BEAM_MOE_ERR_DEVICE_TIMEOUT : BEAM_MOE_OK;
 }
 
+beam_moe_status beam_moe_selftest_wait(void* ws, size_t ws_bytes, int32_t limit_ms,
+                                       void* stream) {
+  if (!ws || ws_bytes < 256 || limit_ms < 1 || limit_ms > 1000) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return BEAM_MOE_ERR_ALIGNMENT;
+  BEAM_CUDA(beam::launch_selftest_wait(static_cast<unsigned*>(ws), limit_ms,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+  return BEAM_MOE_OK;
+}
+
 const char* beam_moe_status_string(beam_moe_status s) {
   switch (s) {
     case BEAM_MOE_OK: return "ok";

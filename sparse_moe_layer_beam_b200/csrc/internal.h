@@ -25,6 +25,7 @@ constexpr uint32_t kFlagProducer = 0x1;
 constexpr uint32_t kFlagMma = 0x2;
 constexpr uint32_t kFlagEpilogue = 0x4;
 constexpr uint32_t kFlagBadExpert = 0x100;
+constexpr uint32_t kFlagSelftest = 0x200;  // beam_moe_selftest_wait's wait ran out
 
 // Byte offsets of every scratch array inside the caller's workspace.
 struct Layout {
@@ -89,6 +90,7 @@ cudaError_t launch_ep_dispatch(const beam_moe_cfg& c, const beam_moe_ep_cfg& g,
                                cudaStream_t st);
 cudaError_t launch_ep_return(const beam_moe_cfg& c, const beam_moe_ep_cfg& g, const EpLayout& P,
                              int64_t rows, void* const* peer_ws, char* ws, cudaStream_t st);
+cudaError_t launch_selftest_wait(unsigned* status, int limit_ms, cudaStream_t st);
 cudaError_t launch_combine_from(const beam_moe_cfg& c, int64_t T, const float* y,
                                 const int32_t* pos, const float* w, uint16_t* out,
                                 cudaStream_t st);

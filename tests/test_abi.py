@@ -158,3 +158,13 @@ def test_host_forward_workspace_and_argument_checks():
     ex = bm.BeamMoeNvfp4Experts(a, a, a, a, 1.0, 1.0, 1.0, 1.0)
     assert L.beam_moe_forward_nvfp4_host(ctypes.byref(odd), 64, a, a, None, ctypes.byref(ex), a,
                                          a, need, None) == UNSUPPORTED
+
+
+def test_selftest_argument_checks():
+    L = bm.lib()
+    a = 1 << 20
+    assert L.beam_moe_selftest_wait(None, 256, 20, None) == INVALID
+    assert L.beam_moe_selftest_wait(a, 255, 20, None) == INVALID
+    assert L.beam_moe_selftest_wait(a, 256, 0, None) == INVALID
+    assert L.beam_moe_selftest_wait(a, 256, 1001, None) == INVALID
+    assert L.beam_moe_selftest_wait(a + 4, 256, 20, None) == ALIGN
