@@ -883,7 +883,6 @@ beam_moe_status beam_moe_ep_experts(const beam_moe_cfg* cfg, const beam_moe_ep_c
   L.counts = P.counts;
   L.offsets = P.offsets;
   L.nb_off = P.nb_off;
-  L.nb2_off = P.nb2_off;
   L.xp = P.recv;
   L.h = P.h;
   int32_t acc = 0;

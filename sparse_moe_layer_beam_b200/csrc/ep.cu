@@ -19,7 +19,7 @@
 // so a peer's buffer is its workspace pointer plus a fixed offset: [status]
 // [receive rows: cap x H x 4 bytes, bf16 on arrival, fp32 y after the down
 // GEMM][return addresses: cap x int32][returned y: T_max K x H fp32][h: cap x
-// I bf16][local expert counts, offsets, token-tile prefixes][routing scratch].
+// I bf16][local expert counts, offsets, token-tile prefix][routing scratch].
 #include <string.h>
 
 #include "internal.h"
@@ -57,7 +57,6 @@ EpLayout make_ep_layout(const beam_moe_cfg& c, const beam_moe_ep_cfg& g) {
   P.counts = take(4 * (size_t)El, 256);
   P.offsets = take(4 * (size_t)(El + 1), 256);
   P.nb_off = take(4 * (size_t)(El + 1), 256);
-  P.nb2_off = take(4 * (size_t)(El + 1), 256);
   P.route = up(o, 1024);
   return P;
 }

@@ -77,7 +77,7 @@ bool nvfp4_pair_supported(const beam_moe_cfg& c);
 // across ranks, so that peers can store into it). `route` is where the
 // routing layout of the rank's own tokens starts.
 struct EpLayout {
-  size_t status, recv, src, yret, h, counts, offsets, nb_off, nb2_off, route;
+  size_t status, recv, src, yret, h, counts, offsets, nb_off, route;
 };
 EpLayout make_ep_layout(const beam_moe_cfg& c, const beam_moe_ep_cfg& g);
 
