@@ -132,12 +132,12 @@ __global__ void __launch_bounds__(128) permute_kernel(const uint16_t* __restrict
       p = chunk_base[(size_t)c * E + e] + rank;
     }
     s_pos[tid] = p;
-    pos[(size_t)t * K + tid] = p;
+    if (blockIdx.y == 0) pos[(size_t)t * K + tid] = p;
   }
   __syncthreads();
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
   const int nv = H / 8;
-  for (int v = tid; v < nv; v += 128) {
+  for (int v = blockIdx.y * 128 + tid; v < nv; v += gridDim.y * 128) {  // this CTA's slice of H
     const uint4 d = __ldg(src + v);
     for (int k = 0; k < K; ++k) {
       const int p = s_pos[k];
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
   __syncthreads();
   const int nv = H / 8;
   uint4* dst = reinterpret_cast<uint4*>(out + (size_t)t * H);
-  for (int v = tid; v < nv; v += 128) {
+  for (int v = blockIdx.y * 128 + tid; v < nv; v += gridDim.y * 128) {  // this CTA's slice of H
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int k = 0; k < K; ++k) {
       const int p = s_pos[k];
@@ -198,7 +198,7 @@ cudaError_t launch_scan(const beam_moe_cfg& c, const Layout& L, char* ws, int32_
 
 cudaError_t launch_permute(const beam_moe_cfg& c, const Layout& L, const uint16_t* x, char* ws,
                            cudaStream_t st) {
-  permute_kernel<<<(unsigned)L.T, 128, 0, st>>>(
+  permute_kernel<<<dim3((unsigned)L.T, (unsigned)h_slices(L.T, c.hidden / 8)), 128, 0, st>>>(
       x, c.hidden, c.top_k, c.n_experts, reinterpret_cast<const int32_t*>(ws + L.ids),
       reinterpret_cast<const int32_t*>(ws + L.chunk_cnt),
       reinterpret_cast<const uint32_t*>(ws + L.chunk_mask), reinterpret_cast<int32_t*>(ws + L.pos),
@@ -208,7 +208,7 @@ cudaError_t launch_permute(const beam_moe_cfg& c, const Layout& L, const uint16_
 
 cudaError_t launch_combine(const beam_moe_cfg& c, const Layout& L, uint16_t* out, char* ws,
                            cudaStream_t st) {
-  combine_kernel<<<(unsigned)L.T, 128, 0, st>>>(
+  combine_kernel<<<dim3((unsigned)L.T, (unsigned)h_slices(L.T, c.hidden / 8)), 128, 0, st>>>(
       reinterpret_cast<const float*>(ws + L.xp), c.hidden, c.top_k,
       reinterpret_cast<const int32_t*>(ws + L.pos), reinterpret_cast<const float*>(ws + L.w), out);
   return cudaGetLastError();
@@ -218,7 +218,8 @@ cudaError_t launch_combine_from(const beam_moe_cfg& c, int64_t T, const float* y
                                 const int32_t* pos, const float* w, uint16_t* out,
                                 cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  combine_kernel<<<(unsigned)T, 128, 0, st>>>(y, c.hidden, c.top_k, pos, w, out);
+  combine_kernel<<<dim3((unsigned)T, (unsigned)h_slices(T, c.hidden / 8)), 128, 0, st>>>(
+      y, c.hidden, c.top_k, pos, w, out);
   return cudaGetLastError();
 }
 

@@ -146,4 +146,13 @@ cudaError_t launch_quantize_rows(int64_t rows, int64_t K, const float* v, float 
 
 int device_sm_count();
 
+// Slices of a token's row that the per-token kernels (permute, combine) spread
+// over a second grid dimension when there are few tokens: enough CTAs for
+// about two per SM, at most one 128-thread pass of `work` items per slice.
+inline int h_slices(int64_t T, int work) {
+  const int64_t want = T > 0 ? (2 * (int64_t)device_sm_count() + T - 1) / T : 1;
+  const int64_t most = (work + 127) / 128;
+  return (int)(want < 1 ? 1 : (want > most ? most : want));
+}
+
 }  // namespace beam

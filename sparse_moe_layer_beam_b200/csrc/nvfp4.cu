@@ -100,11 +100,11 @@ __global__ void __launch_bounds__(128) permute_nvfp4_kernel(
       qp = p - offsets[e] + nb_off[e] * kBN;
     }
     s_q[tid] = qp;
-    pos[(size_t)t * K + tid] = p;
+    if (blockIdx.y == 0) pos[(size_t)t * K + tid] = p;
   }
   __syncthreads();
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
-  for (int b = tid; b < H / 16; b += 128) {
+  for (int b = blockIdx.y * 128 + tid; b < H / 16; b += gridDim.y * 128) {  // this CTA's slice
     const uint4 a = __ldg(src + 2 * b), c = __ldg(src + 2 * b + 1);
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
     float v[16];
@@ -612,7 +612,7 @@ bool nvfp4_supported(const beam_moe_cfg& c) {
 cudaError_t launch_permute_nvfp4(const beam_moe_cfg& c, const Fp4Layout& F, const uint16_t* x,
                                  float gx, char* ws, cudaStream_t st) {
   const Layout& L = F.base;
-  permute_nvfp4_kernel<<<(unsigned)L.T, 128, 0, st>>>(
+  permute_nvfp4_kernel<<<dim3((unsigned)L.T, (unsigned)h_slices(L.T, c.hidden / 16)), 128, 0, st>>>(
       x, c.hidden, c.top_k, c.n_experts, reinterpret_cast<const int32_t*>(ws + L.ids),
       reinterpret_cast<const int32_t*>(ws + L.chunk_cnt),
       reinterpret_cast<const uint32_t*>(ws + L.chunk_mask),

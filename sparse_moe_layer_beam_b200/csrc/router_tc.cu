@@ -29,7 +29,7 @@ namespace {
 constexpr int kRK = 64;          // K per pipeline stage (128 bytes of bf16)
 constexpr int kRThreads = 192;
 constexpr int kRPlaneBytes = kTileM * kRK * 2;  // one plane's 128 x 64 tile
-constexpr int kMaxTcSplit = 32;  // bounds the partial logits the top-k stage reads
+constexpr int kMaxTcSplit = 16;  // bounds the partial logits the top-k stage reads
 
 struct RouterTcParams {
   float* part;   // [n_split][T][E] partial logits
