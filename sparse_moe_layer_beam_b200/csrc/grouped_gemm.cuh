@@ -48,8 +48,16 @@ __device__ __forceinline__ void decode_tile(int tile, const GemmParams& p, int& 
 
 // silu(g) * u in FP32 (fast exponential and division: a few ulp, far below
 // the bf16 rounding of the result).
+// silu(g) u in FP32, with silu(g) = g sigmoid(g) = (g/2)(1 + tanh(g/2)): one
+// hardware tanh (relative error about 2^-11) instead of an exponential and a
+// reciprocal. The error, at most about 2^-11 |g|/2 in silu, stays below the
+// bf16 (or E2M1) rounding that h gets next, and the cheaper epilogue runs
+// the power-capped GEMMs a little faster.
 __device__ __forceinline__ float silu_mul(float g, float u) {
-  return __fdividef(g, 1.0f + __expf(-g)) * u;
+  const float hg = 0.5f * g;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hg));
+  return fmaf(hg, t, hg) * u;
 }
 
 }  // namespace gg
