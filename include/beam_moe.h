@@ -105,8 +105,8 @@ BEAM_MOE_API beam_moe_status beam_moe_route(const beam_moe_cfg* cfg, int64_t T, 
                                void* stream);
 
 /*
- * Routing without any device allocation and without a caller workspace. The
- * paper has no counterpart: this entry point exists for callers that cannot
+ * Routing without any device allocation and without a caller workspace. No
+ * page describes such a call: this entry point exists for callers that cannot
  * call cudaMalloc, for example a serving process whose memory pool has already
  * reserved the GPU's memory for weights and caches, or a runtime that forbids
  * device allocations once it has started. The caller still passes inputs and
