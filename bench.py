@@ -53,13 +53,14 @@ STAGES = ("router_gemm", "router_topk", "scan", "permute", "gateup_gemm", "down_
 KERNELS_PER_STEP = 8
 KERNELS_PER_REPLAY_STEP = 6
 GEMM_SOURCES = ("sparse_moe_layer_beam_b200/csrc/grouped_gemm.cu",
+                "sparse_moe_layer_beam_b200/csrc/grouped_gemm.cuh",
                 "sparse_moe_layer_beam_b200/csrc/sm100.cuh")
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the gate/up
 # kernel per touched expert, from the ncu capture summarised in
 # profiles/grouped_gemm_decode_E32_T8.md; valid only for the decode workload and
 # only while the kernel sources hash to `sources_sha256`.
-GATEUP_TRAFFIC = {"workload": "decode", "bytes_per_touched_expert": 52586103,
-                  "sources_sha256": "17de9080793b81c0f1393c5a0e542a9dc3deab90f1bcd27127c54d109320227d"}
+GATEUP_TRAFFIC = {"workload": "decode", "bytes_per_touched_expert": None,
+                  "sources_sha256": "d2654dc8e6ea4346cb90aa5c6d956b21c8ca1ae00fcb5da28860253f4dd80d0b"}
 
 
 def gemm_sources_sha256():

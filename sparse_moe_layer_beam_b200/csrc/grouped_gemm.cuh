@@ -46,8 +46,6 @@ __device__ __forceinline__ void decode_tile(int tile, const GemmParams& p, int& 
   nb = local - mb * nblk;
 }
 
-// silu(g) * u in FP32 (fast exponential and division: a few ulp, far below
-// the bf16 rounding of the result).
 // silu(g) u in FP32, with silu(g) = g sigmoid(g) = (g/2)(1 + tanh(g/2)): one
 // hardware tanh (relative error about 2^-11) instead of an exponential and a
 // reciprocal. The error, at most about 2^-11 |g|/2 in silu, stays below the

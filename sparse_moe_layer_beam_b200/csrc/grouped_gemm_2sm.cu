@@ -16,6 +16,12 @@
 // a warp's 32 TMEM lanes hold 16 gate rows and the 16 up rows of the same
 // intermediate indices; lanes exchange halves with one shuffle.
 //
+// A CTA loads its half of a tile's token rows as one box of 64 rows when
+// that covers them, else of 128: an expert with up to 128 rows then costs 64
+// rows of operand reads per CTA and k-step, not 128. (Measured: one box per
+// k-step beats an exact cover by several smaller boxes, and 8- to 32-row
+// boxes run slower than the 64-row box although they move fewer bytes.)
+//
 // Roles (both CTAs have the same warps): warp 0 issues this CTA's TMA loads,
 // whose completion is counted on the even CTA's barrier; warp 1 of the even
 // CTA issues the pair's MMAs and commits to barriers in both CTAs; warps 2-5
@@ -41,7 +47,8 @@ constexpr int kPairN = 256;  // max tokens per pair tile (the token block)
 
 struct PairCfg {
   static constexpr int kABytes = 128 * kTileK * 2;  // this CTA's 128 weight rows
-  static constexpr int kBBytes = 128 * kTileK * 2;  // this CTA's half of 256 tokens
+  static constexpr int kBBytes = 128 * kTileK * 2;  // room for this CTA's half of 256 tokens
+  static constexpr int kRowBytes = kTileK * 2;      // one token row of a k-step
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = 6;
   static constexpr int kAccCols = kPairN;  // FP32 accumulator columns per stage
@@ -52,7 +59,8 @@ struct PairCfg {
 template <bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
-                             const __grid_constant__ CUtensorMap tm_x, const GemmParams p) {
+                             const __grid_constant__ CUtensorMap tm_x,
+                             const __grid_constant__ CUtensorMap tm_x64, const GemmParams p) {
   using C = PairCfg;
   constexpr int STAGES = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -85,6 +93,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_x64);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, C::kTmemCols);
@@ -109,8 +118,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         int e, mb, nb;
         decode_tile(tile, p, e, mb, nb);
         const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
-        const int half = ((rows + 15) & ~15) >> 1;
+        const int half = ((rows + 15) & ~15) >> 1;  // 8 .. 128
         const int xrow = __ldg(p.offsets + e) + nb * kPairN + (int)rank * half;
+        const bool box64 = half <= 64;
+        const CUtensorMap* tmx = box64 ? &tm_x64 : &tm_x;
+        const uint32_t stage_tx = 2u * (uint32_t)(C::kABytes + (box64 ? 64 : 128) * C::kRowBytes);
         const int nblk = __ldg(p.nb_off + e + 1) - __ldg(p.nb_off + e);
         const uint64_t pol_w = nblk == 1 ? pol_stream : pol_keep;
         // first weight row of this CTA's 128 (down) or first intermediate
@@ -123,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* sa = smem + stage * C::kStageBytes;
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+          if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx);
           const uint32_t bar = mapa_shared(smem_addr(&full[stage]), 0);
           const int kx = kb * kTileK;
           if (GATEUP) {
@@ -131,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_2d_pair(sa, &tm_w, bar, kx, w0, pol_w);
           }
-          tma_load_2d_pair(sa + C::kABytes, &tm_x, bar, kx, xrow, pol_keep);
+          tma_load_2d_pair(sa + C::kABytes, tmx, bar, kx, xrow, pol_keep);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -256,8 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <bool GATEUP>
-cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p,
-                     cudaStream_t st) {
+cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& tx64,
+                     const GemmParams& p, cudaStream_t st) {
   // Per device: the shared-memory attribute and the number of CTA pairs that
   // can be resident at once (a pair needs two SMs of one GPC). The grid is
   // exactly that many pairs, so no pair waits for another to finish.
@@ -290,7 +302,15 @@ cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const GemmPar
     configured_device = dev;
   }
   cfg.gridDim = dim3((unsigned)(2 * resident_pairs));
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATEUP>, tw, tx, p);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATEUP>, tw, tx, tx64, p);
+}
+
+// Token-row boxes of 128 and 64 rows over the same matrix.
+cudaError_t encode_xmaps(CUtensorMap* m128, CUtensorMap* m64, const void* base, uint64_t cols,
+                         uint64_t rows) {
+  cudaError_t err = encode_tmap_2d_bf16(m128, base, cols, rows, kTileK, 128);
+  if (err != cudaSuccess) return err;
+  return encode_tmap_2d_bf16(m64, base, cols, rows, kTileK, 64);
 }
 
 GemmParams base_params(const beam_moe_cfg& c, const Layout& L, char* ws) {
@@ -312,10 +332,10 @@ bool pair_gemm_supported(const beam_moe_cfg& c) {
 cudaError_t launch_gateup_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w13,
                                char* ws, cudaStream_t st) {
   const int H = c.hidden, I = c.inter, E = c.n_experts;
-  CUtensorMap tw, tx;
+  CUtensorMap tw, tx, tx64;
   cudaError_t err = encode_tmap_w13_interleaved(&tw, w13, (uint64_t)H, (uint64_t)I, (uint64_t)E);
   if (err != cudaSuccess) return err;
-  err = encode_tmap_2d_bf16(&tx, ws + L.xp, (uint64_t)H, (uint64_t)L.A, kTileK, 128);
+  err = encode_xmaps(&tx, &tx64, ws + L.xp, (uint64_t)H, (uint64_t)L.A);
   if (err != cudaSuccess) return err;
   GemmParams p = base_params(c, L, ws);
   p.out = ws + L.h;
@@ -324,16 +344,16 @@ cudaError_t launch_gateup_pair(const beam_moe_cfg& c, const Layout& L, const uin
   p.w_rows = 2 * I;
   p.up_rows = I;
   p.n_mblk = I / 128;  // 128 intermediate indices (gate + up) per pair tile
-  return run_pair<true>(tw, tx, p, st);
+  return run_pair<true>(tw, tx, tx64, p, st);
 }
 
 cudaError_t launch_down_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2,
                              char* ws, cudaStream_t st) {
   const int H = c.hidden, I = c.inter, E = c.n_experts;
-  CUtensorMap tw, tx;
+  CUtensorMap tw, tx, tx64;
   cudaError_t err = encode_tmap_2d_bf16(&tw, w2, (uint64_t)I, (uint64_t)E * H, kTileK, 128);
   if (err != cudaSuccess) return err;
-  err = encode_tmap_2d_bf16(&tx, ws + L.h, (uint64_t)I, (uint64_t)L.A, kTileK, 128);
+  err = encode_xmaps(&tx, &tx64, ws + L.h, (uint64_t)I, (uint64_t)L.A);
   if (err != cudaSuccess) return err;
   GemmParams p = base_params(c, L, ws);
   p.out = ws + L.xp;  // fp32 y reuses the permuted-input rows
@@ -342,7 +362,7 @@ cudaError_t launch_down_pair(const beam_moe_cfg& c, const Layout& L, const uint1
   p.w_rows = H;
   p.up_rows = 0;
   p.n_mblk = H / kPairM;
-  return run_pair<false>(tw, tx, p, st);
+  return run_pair<false>(tw, tx, tx64, p, st);
 }
 
 }  // namespace beam
