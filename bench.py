@@ -59,7 +59,7 @@ GEMM_SOURCES = ("sparse_moe_layer_beam_b200/csrc/grouped_gemm.cu",
 # kernel per touched expert, from the ncu capture summarised in
 # profiles/grouped_gemm_decode_E32_T8.md; valid only for the decode workload and
 # only while the kernel sources hash to `sources_sha256`.
-GATEUP_TRAFFIC = {"workload": "decode", "bytes_per_touched_expert": None,
+GATEUP_TRAFFIC = {"workload": "decode", "bytes_per_touched_expert": 52619897,
                   "sources_sha256": "d2654dc8e6ea4346cb90aa5c6d956b21c8ca1ae00fcb5da28860253f4dd80d0b"}
 
 
