@@ -45,15 +45,32 @@ constexpr int kThreads = 192;
 constexpr int kPairM = 256;  // weight rows per pair tile
 constexpr int kPairN = 256;  // max tokens per pair tile (the token block)
 
+// Tile -> (expert, weight block, token block). An expert's tiles run weight
+// block by weight block, so that each weight tile is read from DRAM once while
+// the expert's token rows stay in L2 - unless the token rows outweigh the
+// weights (more rows than the expert has weight rows): then token block by
+// token block, and the weights are what stays in L2.
+__device__ __forceinline__ void decode_pair_tile(int tile, const GemmParams& p, int& e, int& mb,
+                                                 int& nb) {
+  decode_tile(tile, p, e, mb, nb);
+  if (__ldg(p.counts + e) > p.w_rows) {
+    const int nblk = __ldg(p.nb_off + e + 1) - __ldg(p.nb_off + e);
+    const int local = mb * nblk + nb;
+    nb = local / p.n_mblk;
+    mb = local - nb * p.n_mblk;
+  }
+}
+
 struct PairCfg {
   static constexpr int kABytes = 128 * kTileK * 2;  // this CTA's 128 weight rows
   static constexpr int kBBytes = 128 * kTileK * 2;  // room for this CTA's half of 256 tokens
   static constexpr int kRowBytes = kTileK * 2;      // one token row of a k-step
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = 6;
+  static constexpr int kStages = 7;  // 225 KB of the 227 KB a CTA may use
   static constexpr int kAccCols = kPairN;  // FP32 accumulator columns per stage
   static constexpr int kTmemCols = 512;    // two accumulator stages
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+  static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 limit");
 };
 
 template <bool GATEUP>
@@ -116,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = pair; tile < total && ok; tile += n_pairs) {
         int e, mb, nb;
-        decode_tile(tile, p, e, mb, nb);
+        decode_pair_tile(tile, p, e, mb, nb);
         const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
         const int half = ((rows + 15) & ~15) >> 1;  // 8 .. 128
         const int xrow = __ldg(p.offsets + e) + nb * kPairN + (int)rank * half;
@@ -171,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = pair; tile < total && ok; tile += n_pairs) {
         int e, mb, nb;
-        decode_tile(tile, p, e, mb, nb);
+        decode_pair_tile(tile, p, e, mb, nb);
         const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
         const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32(kPairM, n_mma);
@@ -213,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < total; tile += n_pairs) {
       int e, mb, nb;
-      decode_tile(tile, p, e, mb, nb);
+      decode_pair_tile(tile, p, e, mb, nb);
       const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
       const int n_mma = (rows + 15) & ~15;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, kFlagEpilogue)) break;
