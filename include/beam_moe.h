@@ -292,6 +292,8 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_traced(const beam_moe_cfg* cfg, in
  *   -                       barrier: every rank's dispatch has completed
  *   4 beam_moe_ep_experts   grouped GEMMs over the received rows, each y row
  *                           written back into its source rank's workspace
+ *                           (from the down GEMM's epilogue when it runs on
+ *                           CTA pairs, else by a copy kernel after it)
  *   -                       barrier: every rank's experts call has completed
  *   5 beam_moe_ep_combine   out[t] = sum_k w[t][k] y[t][k], fixed k order
  * No kernel waits for another rank: the caller orders the phases (an NCCL
@@ -355,7 +357,9 @@ BEAM_MOE_API beam_moe_status beam_moe_ep_combine(const beam_moe_cfg* cfg,
  * workspace. *device_flags (may be NULL) receives the raw bits: 0x1 producer,
  * 0x2 MMA issuer, 0x4 epilogue gave up a bounded wait; 0x100 an expert id
  * outside [0, E) reached the dispatch; 0x200 beam_moe_selftest_wait's wait ran
- * out. Returns BEAM_MOE_ERR_DEVICE_TIMEOUT
+ * out; 0x400 a received row's return address named no rank or slot (the row
+ * is not stored; only inconsistent recv_counts lead there). Returns
+ * BEAM_MOE_ERR_DEVICE_TIMEOUT
  * if any bit was set, BEAM_MOE_ERR_CUDA if the stream reports an error.
  */
 BEAM_MOE_API beam_moe_status beam_moe_check(void* ws, size_t ws_bytes, void* stream, uint32_t* device_flags);

@@ -899,9 +899,20 @@ beam_moe_status beam_moe_ep_experts(const beam_moe_cfg* cfg, const beam_moe_ep_c
   BEAM_CUDA(cudaStreamSynchronize(st));  // the host arrays are this call's
   BEAM_CUDA(L.pair_gateup ? beam::launch_gateup_pair(lc, L, w13, w, st)
                           : beam::launch_gateup(lc, L, w13, w, st));
-  BEAM_CUDA(L.pair_down ? beam::launch_down_pair(lc, L, w2, w, st)
-                        : beam::launch_down(lc, L, w2, w, st));
-  BEAM_CUDA(beam::launch_ep_return(*cfg, *ep, P, rows, peer_ws, w, st));
+  if (L.pair_down) {
+    // the down GEMM's epilogue stores every y row into its source's workspace
+    beam::EpReturn ret;
+    memset(&ret, 0, sizeof(ret));
+    ret.src = reinterpret_cast<const int32_t*>(w + P.src);
+    for (int r = 0; r < ep->world; ++r) ret.peer[r] = static_cast<char*>(peer_ws[r]);
+    ret.yret_off = P.yret;
+    ret.world = ep->world;
+    ret.slots = ep->t_max * cfg->top_k;
+    BEAM_CUDA(beam::launch_down_pair(lc, L, w2, w, st, &ret));
+  } else {
+    BEAM_CUDA(beam::launch_down(lc, L, w2, w, st));
+    BEAM_CUDA(beam::launch_ep_return(*cfg, *ep, P, rows, peer_ws, w, st));
+  }
   return BEAM_MOE_OK;
 }
 

@@ -27,8 +27,8 @@
 namespace beam {
 namespace {
 
-constexpr int kMaxWorld = 8;
-constexpr int kSlotBits = 27;  // return address: source rank << 27 | token slot (t K + k)
+constexpr int kMaxWorld = kEpMaxWorld;
+constexpr int kSlotBits = kEpSlotBits;
 
 struct Peers {
   char* ws[kMaxWorld];
@@ -69,7 +69,8 @@ __global__ void __launch_bounds__(128) ep_dispatch_kernel(
     const uint16_t* __restrict__ x, int H, int K, int E, int El, int rank,
     const int32_t* __restrict__ ids, const int32_t* __restrict__ chunk_base,
     const uint32_t* __restrict__ chunk_mask, const int32_t* __restrict__ offsets,
-    const int32_t* __restrict__ send_base, int32_t* __restrict__ pos, Peers peers,
+    const int32_t* __restrict__ send_base, int32_t* __restrict__ pos,
+    const __grid_constant__ Peers peers,
     size_t recv_off, size_t src_off) {
   __shared__ uint16_t* s_dst[32];
   const int t = blockIdx.x;
@@ -107,11 +108,17 @@ __global__ void __launch_bounds__(128) ep_dispatch_kernel(
 __global__ void __launch_bounds__(128) ep_return_kernel(const float* __restrict__ y, int H,
                                                         int64_t rows,
                                                         const int32_t* __restrict__ src,
-                                                        Peers peers, size_t yret_off) {
+                                                        const __grid_constant__ Peers peers,
+                                                        size_t yret_off, int world,
+                                                        int64_t slots, unsigned* status) {
   for (int64_t i = blockIdx.x; i < rows; i += gridDim.x) {
     const uint32_t code = (uint32_t)src[i];
     const int s = (int)(code >> kSlotBits);
     const size_t slot = code & ((1u << kSlotBits) - 1u);
+    if (s >= world || (int64_t)slot >= slots) {  // never stored through
+      if (threadIdx.x == 0) atomicOr(status, kFlagBadReturn);
+      continue;
+    }
     float4* d = reinterpret_cast<float4*>(peers.ws[s] + yret_off) + slot * (H / 4);
     const float4* from = reinterpret_cast<const float4*>(y + (size_t)i * H);
     for (int v = threadIdx.x; v < H / 4; v += 128) d[v] = __ldg(from + v);
@@ -147,7 +154,8 @@ cudaError_t launch_ep_return(const beam_moe_cfg& c, const beam_moe_ep_cfg& g, co
   const int64_t grid = rows < 8L * device_sm_count() ? rows : 8L * device_sm_count();
   ep_return_kernel<<<(unsigned)grid, 128, 0, st>>>(
       reinterpret_cast<const float*>(ws + P.recv), c.hidden, rows,
-      reinterpret_cast<const int32_t*>(ws + P.src), peers, P.yret);
+      reinterpret_cast<const int32_t*>(ws + P.src), peers, P.yret, g.world,
+      g.t_max * c.top_k, reinterpret_cast<unsigned*>(ws + P.status));
   return cudaGetLastError();
 }
 

@@ -4,6 +4,11 @@
 //   gate/up:  [g | u] = W13_e x, h = silu(g) * u in FP32 -> bf16   (K = H)
 //   down:     y = W2_e h -> fp32                                  (K = I)
 //
+// Under expert parallelism the down GEMM's epilogue stores each y row straight
+// into the workspace of the rank the row came from (a peer store over NVLink
+// between GPUs), so the return of y overlaps the tensor-core tiles instead of
+// following them as a copy.
+//
 // One MMA covers 256 weight rows x up to 256 tokens. Each CTA of the pair
 // holds 128 weight rows and half of the tokens in its shared memory and 128
 // accumulator rows in its TMEM, so a CTA moves a third fewer operand bytes per
@@ -29,6 +34,7 @@
 // pair allocates TMEM together and meets at a cluster barrier before freeing
 // it. No load uses multicast. Every wait is bounded.
 #include <cuda_bf16.h>
+#include <string.h>
 
 #include "grouped_gemm.cuh"
 #include "internal.h"
@@ -73,11 +79,14 @@ struct PairCfg {
   static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 limit");
 };
 
-template <bool GATEUP>
+// EPRET: the down GEMM under expert parallelism, storing y rows to their
+// source ranks (a separate instance, so that the plain epilogue stays lean).
+template <bool GATEUP, bool EPRET>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
                              const __grid_constant__ CUtensorMap tm_x,
-                             const __grid_constant__ CUtensorMap tm_x64, const GemmParams p) {
+                             const __grid_constant__ CUtensorMap tm_x64, const GemmParams p,
+                             const __grid_constant__ EpReturn ret) {
   using C = PairCfg;
   constexpr int STAGES = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -257,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               out[(row0 + t) * p.out_ld] = __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(g, u)));
           }
         }
-      } else {
+      } else if (!EPRET) {
         const int col = mb * kPairM + (int)rank * 128 + q * 32 + lane;
         float* out = static_cast<float*>(p.out) + col;
         for (int c0 = 0; c0 < n_mma; c0 += 16) {
@@ -267,6 +276,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (c0 + j < rows) out[(row0 + c0 + j) * p.out_ld] = __uint_as_float(v[j]);
+        }
+      } else {
+        // each row to its source rank's returned-y row of the same slot
+        const int col = mb * kPairM + (int)rank * 128 + q * 32 + lane;
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(tb + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (c0 + j < rows) {
+              const uint32_t code = (uint32_t)__ldg(ret.src + row0 + c0 + j);
+              const int s = (int)(code >> kEpSlotBits);
+              const int64_t slot = code & ((1u << kEpSlotBits) - 1u);
+              if (s < ret.world && slot < ret.slots) {
+                reinterpret_cast<float*>(ret.peer[s] + ret.yret_off)[slot * p.out_ld + col] =
+                    __uint_as_float(v[j]);
+              } else if (lane == 0) {  // never stored through
+                atomicOr(p.status, kFlagBadReturn);
+              }
+            }
+          }
         }
       }
       tc_fence_before();
@@ -284,9 +315,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool GATEUP>
+template <bool GATEUP, bool EPRET>
 cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& tx64,
-                     const GemmParams& p, cudaStream_t st) {
+                     const GemmParams& p, const EpReturn& ret, cudaStream_t st) {
   // Per device: the shared-memory attribute and the number of CTA pairs that
   // can be resident at once (a pair needs two SMs of one GPC). The grid is
   // exactly that many pairs, so no pair waits for another to finish.
@@ -307,19 +338,19 @@ cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const CUtenso
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (configured_device != dev) {
-    err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATEUP>,
+    err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATEUP, EPRET>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::kSmemBytes);
     if (err != cudaSuccess) return err;
     cfg.gridDim = dim3((unsigned)(device_sm_count() & ~1));
     int clusters = 0;
-    err = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<GATEUP>, &cfg);
+    err = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<GATEUP, EPRET>, &cfg);
     if (err != cudaSuccess) return err;
     if (clusters < 1) return cudaErrorInvalidConfiguration;
     resident_pairs = clusters < device_sm_count() / 2 ? clusters : device_sm_count() / 2;
     configured_device = dev;
   }
   cfg.gridDim = dim3((unsigned)(2 * resident_pairs));
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATEUP>, tw, tx, tx64, p);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATEUP, EPRET>, tw, tx, tx64, p, ret);
 }
 
 // Token-row boxes of 128 and 64 rows over the same matrix.
@@ -361,11 +392,13 @@ cudaError_t launch_gateup_pair(const beam_moe_cfg& c, const Layout& L, const uin
   p.w_rows = 2 * I;
   p.up_rows = I;
   p.n_mblk = I / 128;  // 128 intermediate indices (gate + up) per pair tile
-  return run_pair<true>(tw, tx, tx64, p, st);
+  EpReturn none;
+  memset(&none, 0, sizeof(none));
+  return run_pair<true, false>(tw, tx, tx64, p, none, st);
 }
 
 cudaError_t launch_down_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2,
-                             char* ws, cudaStream_t st) {
+                             char* ws, cudaStream_t st, const EpReturn* ret) {
   const int H = c.hidden, I = c.inter, E = c.n_experts;
   CUtensorMap tw, tx, tx64;
   cudaError_t err = encode_tmap_2d_bf16(&tw, w2, (uint64_t)I, (uint64_t)E * H, kTileK, 128);
@@ -379,7 +412,10 @@ cudaError_t launch_down_pair(const beam_moe_cfg& c, const Layout& L, const uint1
   p.w_rows = H;
   p.up_rows = 0;
   p.n_mblk = H / kPairM;
-  return run_pair<false>(tw, tx, tx64, p, st);
+  if (ret && ret->src) return run_pair<false, true>(tw, tx, tx64, p, *ret, st);
+  EpReturn none;
+  memset(&none, 0, sizeof(none));
+  return run_pair<false, false>(tw, tx, tx64, p, none, st);
 }
 
 }  // namespace beam

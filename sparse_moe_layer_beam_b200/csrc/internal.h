@@ -26,6 +26,7 @@ constexpr uint32_t kFlagMma = 0x2;
 constexpr uint32_t kFlagEpilogue = 0x4;
 constexpr uint32_t kFlagBadExpert = 0x100;
 constexpr uint32_t kFlagSelftest = 0x200;  // beam_moe_selftest_wait's wait ran out
+constexpr uint32_t kFlagBadReturn = 0x400; // a received row's return address out of range
 
 // Byte offsets of every scratch array inside the caller's workspace.
 struct Layout {
@@ -76,6 +77,22 @@ bool nvfp4_pair_supported(const beam_moe_cfg& c);
 // Expert parallelism: byte offsets inside every rank's workspace (identical
 // across ranks, so that peers can store into it). `route` is where the
 // routing layout of the rank's own tokens starts.
+// Expert parallelism: a received row's return address is its source rank
+// << kEpSlotBits | its token slot (t K + k) on that rank.
+constexpr int kEpMaxWorld = 8;
+constexpr int kEpSlotBits = 27;
+
+// Where the down GEMM on CTA pairs stores y. src == nullptr: the workspace's
+// y rows. Otherwise each row goes straight to its source rank's returned-y
+// buffer, peer[rank] + yret_off + slot * H floats (a peer store).
+struct EpReturn {
+  const int32_t* src;        // [rows] return address of every received row
+  char* peer[kEpMaxWorld];   // every rank's workspace
+  size_t yret_off;           // the returned-y buffer inside a workspace
+  int world;                 // ranks; a return address names one of them
+  int64_t slots;             // returned-y rows per rank (T_max K)
+};
+
 struct EpLayout {
   size_t status, recv, src, yret, h, counts, offsets, nb_off, route;
 };
@@ -118,7 +135,7 @@ bool pair_gemm_supported(const beam_moe_cfg& c);
 cudaError_t launch_gateup_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w13,
                                char* ws, cudaStream_t st);
 cudaError_t launch_down_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2,
-                             char* ws, cudaStream_t st);
+                             char* ws, cudaStream_t st, const EpReturn* ret = nullptr);
 cudaError_t launch_combine(const beam_moe_cfg& c, const Layout& L, uint16_t* out, char* ws,
                            cudaStream_t st);
 cudaError_t launch_copy_routes(const beam_moe_cfg& c, const Layout& L, int32_t* ids_out,

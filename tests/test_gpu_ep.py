@@ -75,5 +75,13 @@ def test_ep_tiny(world, Ts):
     _check(synth.workload("tiny"), world, Ts)
 
 
+@pytest.mark.parametrize("world,Ts", [(2, [900, 600]), (4, [700, 5, 500, 300])])
+def test_ep_tiny_many_rows(world, Ts):
+    """Hundreds of rows per local expert: the down GEMM runs on CTA pairs and
+    its epilogue stores every y row straight into the source rank's
+    workspace (no separate return pass)."""
+    _check(synth.workload("tiny"), world, Ts)
+
+
 def test_ep_decode_full_size_eight_ranks():  # 32 experts per rank, 64 tokens each
     _check(synth.workload("decode"), 8, [64] * 8, n_sample=12)
