@@ -326,7 +326,7 @@ BEAM_MOE_API beam_moe_status beam_moe_ep_route(const beam_moe_cfg* cfg, const be
  * order; sources follow one another in rank order). recv_counts [E/world]
  * int32 (host, out): rows this rank receives per local expert; *recv_rows
  * their sum. Fails with BEAM_MOE_ERR_WORKSPACE_TOO_SMALL if any rank would
- * receive more than recv_cap rows (every rank reaches the same verdict). */
+ * receive more than recv_cap rows (every rank reaches the same result). */
 BEAM_MOE_API beam_moe_status beam_moe_ep_plan(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep,
                                               const int32_t* counts_all, int32_t* send_base,
                                               int32_t* recv_counts, int64_t* recv_rows);
