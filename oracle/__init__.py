@@ -45,6 +45,8 @@ def lib():
         L.oracle_e2m1_encode.argtypes = [ctypes.c_float]
         L.oracle_nvfp4_quantize.restype = ctypes.c_int
         L.oracle_nvfp4_quantize.argtypes = [P, ctypes.c_int64, ctypes.c_float, P, P]
+        L.oracle_nvfp4_value.restype = ctypes.c_double
+        L.oracle_nvfp4_value.argtypes = [P, P, ctypes.c_int64, ctypes.c_double]
         L.oracle_experts_nvfp4.restype = ctypes.c_int
         L.oracle_experts_nvfp4.argtypes = [ctypes.POINTER(OracleCfg), ctypes.c_int64, P, P, P, P,
                                            P, P, P, ctypes.c_double, ctypes.c_double,
@@ -171,6 +173,15 @@ def nvfp4_quantize(values, g):
         if rc != 0:
             raise ValueError(f"oracle_nvfp4_quantize failed ({rc})")
     return codes, sf
+
+
+def nvfp4_values(codes, sf, g):
+    """One row (codes [K/2], scales [K/16]) -> fp64 values [K] through the C
+    decoder the expert path uses (element by element)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    return np.array([lib().oracle_nvfp4_value(codes.ctypes.data, sf.ctypes.data, i, g)
+                     for i in range(2 * codes.size)])
 
 
 _E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])

@@ -79,6 +79,21 @@ def test_packing_order_low_nibble_first():
     assert codes[0, 0] == (7 | (0xD << 4)) and codes[0, 7] == (2 << 4)
 
 
+def test_decoder_reads_the_packing_order():
+    """The C decoder the expert path uses reads element 2i from the low nibble
+    and 2i+1 from the high one, with the block's scale: it returns the packed
+    grid values in order. (A decoder that swapped the nibbles would leave every
+    dot product of the expert path unchanged, since it would permute both
+    operands alike, so it is pinned here on its own.)"""
+    v = np.zeros((1, 32), np.float32)
+    v[0, 0], v[0, 1], v[0, 2], v[0, 15] = 6.0, -3.0, 0.5, 1.0
+    v[0, 16], v[0, 17] = -3.0, 12.0  # second block: scale 2, values on its grid
+    codes, sf = oracle.nvfp4_quantize(v, np.float32(1.0))
+    dec = oracle.nvfp4_values(codes[0], sf[0], 1.0)
+    assert np.array_equal(dec, v[0].astype(np.float64))
+    assert np.array_equal(dec, oracle.nvfp4_dequant(codes, sf, 1.0)[0])
+
+
 def _swiglu_nvfp4_numpy(x_bits, c13, s13, c2, s2, gw, gx, gh):
     """Numpy float64 matmuls on dequantised values; activations quantised with
     the oracle's (separately pinned) quantiser."""
