@@ -15,7 +15,11 @@ from tests import _gpu, _inputs
 pytestmark = pytest.mark.gpu
 
 
-def ep_forward(wl, xs, world, bias=None):
+def ep_forward(wl, xs, world, bias=None, fill=None, extra_rows=0):
+    """The five phases over emulated ranks. fill: a byte every workspace holds
+    before the first call (its status word excepted); extra_rows: rows each
+    owner is told its last local expert received beyond what was dispatched.
+    Returns (outputs, counts_all, plans, status bits of every rank)."""
     cfg = _gpu.cfg_of(wl)
     w13, w2, wr = _gpu.device_weights(wl)
     El, H = wl.E // world, wl.H
@@ -24,6 +28,10 @@ def ep_forward(wl, xs, world, bias=None):
     eps = [bm.ep_cfg(world, r, max(Ts), cap) for r in range(world)]
     wss = [torch.empty(bm.beam_moe_ep_workspace_size(cfg, ep), dtype=torch.uint8, device="cuda")
            for ep in eps]
+    if fill is not None:
+        for ws in wss:
+            ws.fill_(fill)
+            ws[:256].zero_()  # the status word
     peers = [ws.data_ptr() for ws in wss]
     xd = [_gpu.to_dev_bits(x) if x.shape[0] else torch.empty((0, H), dtype=torch.int16,
                                                               device="cuda") for x in xs]
@@ -39,7 +47,9 @@ def ep_forward(wl, xs, world, bias=None):
     torch.cuda.synchronize()  # barrier: every dispatch has landed
     w13_bytes, w2_bytes = 2 * wl.I * wl.H * 2, wl.H * wl.I * 2  # one expert's weights
     for r in range(world):
-        bm.beam_moe_ep_experts(cfg, eps[r], plans[r][1], w13.data_ptr() + r * El * w13_bytes,
+        recv = plans[r][1].copy()
+        recv[-1] += extra_rows
+        bm.beam_moe_ep_experts(cfg, eps[r], recv, w13.data_ptr() + r * El * w13_bytes,
                                w2.data_ptr() + r * El * w2_bytes, peers, wss[r])
     torch.cuda.synchronize()  # barrier: every y row is back at its source
     outs = []
@@ -47,16 +57,15 @@ def ep_forward(wl, xs, world, bias=None):
         out = torch.empty((Ts[r], H), dtype=torch.int16, device="cuda")
         bm.beam_moe_ep_combine(cfg, eps[r], Ts[r], out, wss[r])
         outs.append(_gpu.bits_of(out))
-    for ws in wss:
-        assert bm.beam_moe_check(ws) == 0
-    return outs, counts_all, plans
+    return outs, counts_all, plans, [bm.beam_moe_check(ws) for ws in wss]
 
 
-def _check(wl, world, Ts, n_sample=None):
+def _check(wl, world, Ts, n_sample=None, fill=None, extra_rows=0, want_flags=0):
     T = sum(Ts)
     x, _, wr, b, r = _inputs.routed_inputs(wl.with_T(T))
     xs = np.split(x, np.cumsum(Ts)[:-1])
-    outs, counts_all, plans = ep_forward(wl, xs, world, b)
+    outs, counts_all, plans, flags = ep_forward(wl, xs, world, b, fill, extra_rows)
+    assert flags == [want_flags] * world
     assert sum(p[2] for p in plans) == T * wl.K  # every assignment received once
     got = np.concatenate(outs)
     tokens = np.arange(T) if n_sample is None else synth.sample_tokens(T, n_sample)
@@ -85,3 +94,15 @@ def test_ep_tiny_many_rows(world, Ts):
 
 def test_ep_decode_full_size_eight_ranks():  # 32 experts per rank, 64 tokens each
     _check(synth.workload("decode"), 8, [64] * 8, n_sample=12)
+
+
+@pytest.mark.parametrize("Ts", [[900, 600], [100, 37]])
+def test_ep_return_address_out_of_range_is_dropped_and_flagged(Ts):
+    """Each owner is told its last local expert received 16 rows more than any
+    rank dispatched. Their return addresses keep the workspace's 0xFF fill,
+    which names no rank, so the experts phase computes those rows but stores
+    none of them, and sets status bit 0x400. Both return paths are covered:
+    the pair down GEMM's own stores ([900, 600]) and the copy after the 1-CTA
+    GEMM ([100, 37]). Every access stays inside the workspaces, and the real
+    rows' outputs still match the oracle."""
+    _check(synth.workload("tiny"), 2, Ts, fill=0xFF, extra_rows=16, want_flags=0x400)
