@@ -80,6 +80,21 @@ def gateup_traffic(wl, touched):
     return rec["bytes_per_touched_expert"] * touched
 
 
+def host_chunking(T, nvfp4):
+    """How the host-buffer entry points split T tokens (the rule of
+    include/beam_moe.h, BEAM_MOE_HOST_CHUNK): one chunk below two chunks'
+    worth, else chunks of BEAM_MOE_HOST_CHUNK, twice that for bf16 batches of
+    at least eight."""
+    import sparse_moe_layer_beam_b200 as bm  # constants only; the library loads on first call
+
+    c = bm.HOST_CHUNK
+    if T < 2 * c:
+        return "one chunk"
+    size = 2 * c if (not nvfp4 and T >= 8 * c) else c
+    n = -(-T // size)
+    return f"{n} chunks of {size} tokens, copies overlapped"
+
+
 def describe(wl):
     extra = ""
     if wl.n_hot:
@@ -460,7 +475,7 @@ def run_ours(args, wl):
                 "d2h_bytes_per_step": wl.T * wl.H * 2,
                 "call": ("copies around beam_moe_forward_routed" if args.replay else
                          ("beam_moe_forward_nvfp4_host" if nvfp4 else "beam_moe_forward_host")
-                         + " (chunked from 16384 tokens, copies overlapped)")},
+                         + f" ({host_chunking(wl.T, nvfp4)})")},
         "gpu_launches": (KERNELS_PER_REPLAY_STEP if args.replay else KERNELS_PER_STEP)
         * args.steps,
         "clocks": clk,

@@ -168,3 +168,29 @@ def test_selftest_argument_checks():
     assert L.beam_moe_selftest_wait(a, 256, 0, None) == INVALID
     assert L.beam_moe_selftest_wait(a, 256, 1001, None) == INVALID
     assert L.beam_moe_selftest_wait(a + 4, 256, 20, None) == ALIGN
+
+
+def test_bench_describes_the_host_chunking_the_library_plans():
+    """bench.py's e2e line names how the host-buffer call splits a batch. The
+    library's host workspace is one forward's workspace (of the larger of a
+    full and the last chunk) plus two staging buffers (upload and download)
+    per chunk in flight, so its size pins the chunking the description states."""
+    import bench
+
+    def up(v):
+        return (v + 1023) // 1024 * 1024
+
+    cfg = bm.beam_cfg()
+    for T, nvfp4 in [(64, False), (4096, True), (16384, False), (20000, False),
+                     (65536, False), (65536, True)]:
+        desc = bench.host_chunking(T, nvfp4)
+        size = T if desc == "one chunk" else int(desc.split(" of ")[1].split()[0])
+        n = -(-T // size)
+        if desc != "one chunk":
+            assert desc.startswith(f"{n} chunks")
+        fwd_op = bm.OP_FORWARD_NVFP4 if nvfp4 else bm.OP_FORWARD
+        host_op = bm.OP_FORWARD_NVFP4_HOST if nvfp4 else bm.OP_FORWARD_HOST
+        last = T - (n - 1) * size
+        fwd = up(max(ws_size(cfg, size, fwd_op)[1], ws_size(cfg, last, fwd_op)[1]))
+        bufs = 1 if n == 1 else 2
+        assert ws_size(cfg, T, host_op) == (OK, fwd + 2 * bufs * up(size * cfg.hidden * 2))
