@@ -137,6 +137,50 @@ def algorithmic(wl, counts, fmt="bf16"):
     }
 
 
+def roofline(alg, gate_ms, ms_step, peaks, peak_kind, nvfp4):
+    """The line's `roofline` (the gate/up kernel) and `block` objects.
+
+    gate_ms: the gate/up kernel's mean event time (None when the entry point
+    records no per-stage events). The tensor peak is the burst figure for
+    steps under 10 ms and the sustained (power-capped) one from 10 ms on; for
+    NVFP4 it is 4 x the measured bf16 peak (the nominal dense FP4:BF16 ratio).
+    The kernel's bound follows from its algorithmic bytes and flops: whichever
+    takes longer at its peak."""
+    if nvfp4:
+        peaks = dict(peaks, bf16_tflops=4 * peaks["bf16_tflops"],
+                     bf16_tflops_sustained=4 * peaks.get("bf16_tflops_sustained",
+                                                         peaks["bf16_tflops"]))
+    sustained = ms_step >= 10.0 and "bf16_tflops_sustained" in peaks
+    tc_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    t_hbm = alg["gateup_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = alg["gateup_flops"] / (tc_peak * 1e12)
+    ok = gate_ms is not None and gate_ms == gate_ms and gate_ms > 0
+    if t_hbm >= t_tc:
+        achieved = alg["gateup_bytes"] / (gate_ms / 1000.0) / 1e9 if ok else None
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = alg["gateup_flops"] / (gate_ms / 1000.0) / 1e12 if ok else None
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                "peak_kind": "sustained" if sustained else "burst"}
+    roof["frac"] = None if roof["achieved"] is None else roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["algorithmic_bytes"] = alg["gateup_bytes"]
+    roof["kernel"] = "gateup_grouped_gemm_nvfp4" if nvfp4 else "gateup_grouped_gemm"
+    if nvfp4:
+        roof["peak_note"] = "dense FP4 tensor peak = 4 x measured bf16 (nominal ratio)"
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
+        else "fallback"
+    block_s = ms_step / 1000.0
+    block = {"hbm_gbs": alg["block_bytes"] / block_s / 1e9,
+             "hbm_frac": alg["block_bytes"] / block_s / 1e9 / peaks["hbm_gbs"],
+             "tflops": alg["expert_flops"] / block_s / 1e12,
+             "tensor_frac": alg["expert_flops"] / block_s / 1e12 / tc_peak,
+             "tensor_frac_of_burst": alg["expert_flops"] / block_s / 1e12 / peaks["bf16_tflops"],
+             "tensor_peak_kind": "sustained" if sustained else "burst",
+             "touched_experts": alg["touched_experts"]}
+    return roof, block
+
+
 class ClockSampler:
     """nvidia-smi samples of clocks and throttle reasons during the timed region."""
 
@@ -417,39 +461,12 @@ def run_ours(args, wl):
 
     alg = algorithmic(wl, counts.cpu().numpy(), args.format)
     peaks, peak_kind = load_peaks()
-    if nvfp4:  # dense FP4 = 4x dense BF16 (nominal 9 vs 2.25 PFLOP/s), scaled from the measured
-        peaks = dict(peaks, bf16_tflops=4 * peaks["bf16_tflops"],
-                     bf16_tflops_sustained=4 * peaks.get("bf16_tflops_sustained",
-                                                         peaks["bf16_tflops"]))
-    # Tensor peak: the burst figure for short steps, the sustained (power-capped)
-    # figure once a step lasts 10 ms or more and the GPU runs at its power cap.
-    sustained = ms_step >= 10.0 and "bf16_tflops_sustained" in peaks
-    tc_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     stage_mean = {n: float(stage_ms[:, i].mean()) for i, n in enumerate(STAGES)}
-    # the gate/up grouped GEMM dominates every configuration; its bound follows
-    # from its arithmetic intensity (flop per weight byte = rows per expert)
     gate_ms = float(stage_ms[:, 4].mean()) if trace is not None else float("nan")
-    t_hbm = alg["gateup_bytes"] / (peaks["hbm_gbs"] * 1e9)
-    t_tc = alg["gateup_flops"] / (tc_peak * 1e12)
-    if t_hbm >= t_tc:
-        achieved = alg["gateup_bytes"] / (gate_ms / 1000.0) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-    else:
-        achieved = alg["gateup_flops"] / (gate_ms / 1000.0) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                "peak_kind": "sustained" if sustained else "burst"}
-    if args.replay:  # no per-stage events on this entry point
-        roof.update(achieved=None, frac=None)
-    roof["frac"] = None if roof["achieved"] is None else roof["achieved"] / roof["peak"]
+    roof, block = roofline(alg, None if args.replay else gate_ms, ms_step, peaks, peak_kind,
+                           nvfp4)
     # the recorded DRAM traffic belongs to the bf16 gate/up kernel only
     roof["traffic"] = None if nvfp4 else gateup_traffic(wl, alg["touched_experts"])
-    roof["algorithmic_bytes"] = alg["gateup_bytes"]
-    roof["kernel"] = "gateup_grouped_gemm_nvfp4" if nvfp4 else "gateup_grouped_gemm"
-    if nvfp4:
-        roof["peak_note"] = "dense FP4 tensor peak = 4 x measured bf16 (nominal ratio)"
-    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
-        else "fallback"
-    block_s = ms_step / 1000.0
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -462,14 +479,7 @@ def run_ours(args, wl):
                    "l2": "flushed before every timed step (256 MB write, outside the events)",
                    "parallelism": f"replicas x{world} (token data parallel, no exchange)"},
         "roofline": roof,
-        "block": {"hbm_gbs": alg["block_bytes"] / block_s / 1e9,
-                  "hbm_frac": alg["block_bytes"] / block_s / 1e9 / peaks["hbm_gbs"],
-                  "tflops": alg["expert_flops"] / block_s / 1e12,
-                  "tensor_frac": alg["expert_flops"] / block_s / 1e12 / tc_peak,
-                  "tensor_frac_of_burst": alg["expert_flops"] / block_s / 1e12
-                  / peaks["bf16_tflops"],
-                  "tensor_peak_kind": "sustained" if sustained else "burst",
-                  "touched_experts": alg["touched_experts"]},
+        "block": block,
         "stages_ms": None if args.replay else stage_mean,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * wl.H * 2,
                 "d2h_bytes_per_step": wl.T * wl.H * 2,
