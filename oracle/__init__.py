@@ -35,6 +35,8 @@ def lib():
         L.oracle_swiglu_expert.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, P, P]
         L.oracle_experts.restype = ctypes.c_int
         L.oracle_experts.argtypes = [ctypes.POINTER(OracleCfg), ctypes.c_int64, P, P, P, P, P, P]
+        L.oracle_hidden.restype = ctypes.c_int
+        L.oracle_hidden.argtypes = [ctypes.POINTER(OracleCfg), ctypes.c_int64, P, P, P, P]
         L.oracle_e2m1_value.restype = ctypes.c_double
         L.oracle_e2m1_value.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_value.restype = ctypes.c_double
@@ -130,6 +132,27 @@ def experts(cfg, x_bits, ids, weights, w13_of, w2_of):
                               _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle_experts failed ({rc})")
+    return out
+
+
+def hidden(cfg, x_bits, ids, w13_of):
+    """a [T, K, I] fp64: silu(Wg x_t) * (Wu x_t) of every routed (token, expert)
+    pair, the gate/up step's output before the down projection."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T = x.shape[0]
+    E = cfg.n_experts
+    keep = []
+    p13 = (ctypes.c_void_p * E)()
+    for e in np.unique(ids):
+        a = np.ascontiguousarray(w13_of[int(e)], dtype=np.uint16)
+        assert a.shape == (2 * cfg.inter, cfg.hidden)
+        keep.append(a)
+        p13[int(e)] = a.ctypes.data
+    out = np.zeros((T, cfg.top_k, cfg.inter))
+    rc = lib().oracle_hidden(ctypes.byref(cfg), T, _ptr(x), _ptr(ids), p13, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_hidden failed ({rc})")
     return out
 
 

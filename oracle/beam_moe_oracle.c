@@ -146,11 +146,8 @@ int oracle_route(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const floa
   return bad ? -2 : 0;
 }
 
-int oracle_swiglu_expert(int32_t H, int32_t I, const double* x, const uint16_t* w13,
-                         const uint16_t* w2, double* y) {
-  if (H <= 0 || I <= 0 || !x || !w13 || !w2 || !y) return -1;
-  double* a = (double*)malloc(sizeof(double) * (size_t)I);
-  if (!a) return -2;
+/* a = silu(Wg x) * (Wu x) for one token: the expert's hidden activations. */
+static void swiglu_hidden(int32_t H, int32_t I, const double* x, const uint16_t* w13, double* a) {
   for (int i = 0; i < I; ++i) {
     const uint16_t* wg = w13 + (int64_t)i * H;
     const uint16_t* wu = w13 + (int64_t)(I + i) * H;
@@ -161,6 +158,14 @@ int oracle_swiglu_expert(int32_t H, int32_t I, const double* x, const uint16_t* 
     }
     a[i] = g / (1.0 + exp(-g)) * u; /* silu(g) * u */
   }
+}
+
+int oracle_swiglu_expert(int32_t H, int32_t I, const double* x, const uint16_t* w13,
+                         const uint16_t* w2, double* y) {
+  if (H <= 0 || I <= 0 || !x || !w13 || !w2 || !y) return -1;
+  double* a = (double*)malloc(sizeof(double) * (size_t)I);
+  if (!a) return -2;
+  swiglu_hidden(H, I, x, w13, a);
   for (int j = 0; j < H; ++j) {
     const uint16_t* wd = w2 + (int64_t)j * I;
     double acc = 0.0;
@@ -169,6 +174,39 @@ int oracle_swiglu_expert(int32_t H, int32_t I, const double* x, const uint16_t* 
   }
   free(a);
   return 0;
+}
+
+int oracle_hidden(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const int32_t* ids,
+                  const uint16_t* const* w13, double* a) {
+  if (!cfg_ok(cfg) || T < 0) return -1;
+  if (T == 0) return 0;
+  if (!x || !ids || !w13 || !a) return -1;
+  const int H = cfg->hidden, I = cfg->inter, E = cfg->n_experts, K = cfg->top_k;
+  int bad = 0;
+#pragma omp parallel
+  {
+    double* xd = (double*)malloc(sizeof(double) * (size_t)H);
+    if (!xd) {
+#pragma omp atomic write
+      bad = -2;
+    } else {
+#pragma omp for schedule(dynamic, 1)
+      for (int64_t t = 0; t < T; ++t) {
+        for (int h = 0; h < H; ++h) xd[h] = bf16_to_double(x[t * (int64_t)H + h]);
+        for (int k = 0; k < K; ++k) {
+          const int e = ids[t * K + k];
+          if (e < 0 || e >= E || !w13[e]) {
+#pragma omp atomic write
+            bad = -3;
+            continue;
+          }
+          swiglu_hidden(H, I, xd, w13[e], a + (t * K + k) * (int64_t)I);
+        }
+      }
+    }
+    free(xd);
+  }
+  return bad;
 }
 
 int oracle_experts(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const int32_t* ids,

@@ -74,6 +74,15 @@ int oracle_swiglu_expert(int32_t H, int32_t I, const double* x, const uint16_t* 
                          const uint16_t* w2, double* y);
 
 /*
+ * The hidden activations of every routed (token, expert) pair, the quantity
+ * the gate/up step produces before the down projection:
+ *   a[t][k][i] = silu(Wg_e x_t)[i] * (Wu_e x_t)[i],   e = ids[t][k]    (fp64 [T][K][I])
+ * w13[e] as for oracle_experts; w2 is not needed.
+ */
+int oracle_hidden(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const int32_t* ids,
+                  const uint16_t* const* w13, double* a);
+
+/*
  * Expert path and combine for T tokens given their routes:
  *   out[t] = sum_k weights[t][k] * expert_{ids[t][k]}(x[t])     (fp64 [T][H])
  * w13[e] / w2[e] point to expert e's weights; an expert no token selects may

@@ -65,6 +65,15 @@ MUTANTS = [
     ("NVFP4 nibble order", [
         ("uint8_t code = (i & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);",
          "uint8_t code = (i & 1) ? (uint8_t)(byte & 15) : (uint8_t)(byte >> 4);")]),
+    ("expert margin over every group", [
+        ("if (gkept[e / per] && !taken[e] && c[e] > bestu) bestu = c[e];",
+         "if (!taken[e] && c[e] > bestu) bestu = c[e];")]),
+    ("group margin from the best kept group", [
+        ("if (gkept[g] && gs[g] < lastk) lastk = gs[g];",
+         "if (gkept[g] && (lastk == INFINITY || gs[g] > lastk)) lastk = gs[g];")]),
+    ("hidden activations in the wrong slot", [
+        ("swiglu_hidden(H, I, xd, w13[e], a + (t * K + k) * (int64_t)I);",
+         "swiglu_hidden(H, I, xd, w13[e], a + t * (int64_t)I);")]),
     ("NVFP4 h not quantised", [
         ("for (int i = 0; i < I; ++i) ad[i] = oracle_nvfp4_value(ac, as, i, (double)g_h);",
          "for (int i = 0; i < I; ++i) ad[i] = af[i];")]),
@@ -80,6 +89,8 @@ PINS = [
     ("test_oracle_pins", "test_scores_are_sigmoid_of_router_logits", ()),
     ("test_oracle_pins", "test_bias_on_logits_and_selection_only_bias", ()),
     ("test_oracle_pins", "test_single_expert_is_dense_swiglu", ()),
+    ("test_oracle_pins", "test_hidden_is_dense_swiglu_hidden", ()),
+    ("test_oracle_pins", "test_margins_match_an_independent_recomputation", ("tiny", 0)),
     ("test_oracle_pins", "test_identical_experts_closed_form", (True,)),
     ("test_oracle_pins", "test_identical_experts_closed_form", (False,)),
     ("test_oracle_pins", "test_expert_index_closed_form", ()),

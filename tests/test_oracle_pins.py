@@ -133,6 +133,48 @@ def test_invariants_at_beam_shape():
     assert r["margins"].min() >= _inputs.MARGIN
 
 
+def _margins_numpy(s, choice, G, Gk, K):
+    """(group margin, expert margin) of one token from the scores alone: rank
+    the groups by the sum of their two best choice scores, keep Gk, take the K
+    best choice scores among the kept groups' experts; each margin is the last
+    kept candidate's value minus the best rejected one's (inf if none)."""
+    E = s.shape[0]
+    per = E // G
+    gscore = np.sort(choice.reshape(G, per), axis=1)[:, -2:].sum(axis=1)
+    order = sorted(range(G), key=lambda g: (-gscore[g], g))
+    kept, rest = order[:Gk], order[Gk:]
+    mg = gscore[kept].min() - gscore[rest].max() if rest else math.inf
+    eligible = np.concatenate([np.arange(g * per, (g + 1) * per) for g in kept])
+    ranked = sorted(eligible.tolist(), key=lambda e: (-choice[e], e))
+    me = choice[ranked[K - 1]] - choice[ranked[K]] if len(ranked) > K else math.inf
+    return mg, me
+
+
+@pytest.mark.parametrize("name,bias_mode", [("tiny", 0), ("tiny", 1), ("decode", 0)])
+def test_margins_match_an_independent_recomputation(name, bias_mode):
+    """The margins the parity inputs are re-drawn on, recomputed from sigmoid
+    scores of numpy logits, with the group and expert ranking written out
+    here: a margin taken from the wrong side, over the wrong experts or from
+    the wrong kept group would let near-tie tokens into the parity tests."""
+    wl = synth.workload(name).with_T(48)
+    x = synth.host_x(wl)
+    wr = synth.host_router(wl)
+    bias = np.linspace(-0.2, 0.2, wl.E).astype(np.float32)
+    r = oracle.route(oracle.cfg_for(wl, bias_mode=bias_mode), x, wr, bias)
+    lg = f64(x) @ wr.astype(np.float64).T
+    for t in range(wl.T):
+        if bias_mode == 0:
+            s = expit(lg[t] + bias)
+            c = s
+        else:
+            s = expit(lg[t])
+            c = s + bias.astype(np.float64)
+        mg, me = _margins_numpy(s, c, wl.G, wl.Gk, wl.K)
+        assert r["margins"][t, 0] == pytest.approx(mg, rel=1e-9, abs=1e-12), t
+        assert r["margins"][t, 1] == pytest.approx(me, rel=1e-9, abs=1e-12), t
+    assert r["margins"].min() >= 0.0
+
+
 def test_tie_case_selects_lowest_indices():
     for name in ("tiny", "decode"):
         wl = synth.workload(name).with_T(4)
@@ -191,6 +233,21 @@ def test_single_expert_is_dense_swiglu():
     ref = dense_swiglu(x, w13, w2)
     for t in range(4):
         assert np.allclose(oracle.swiglu_expert(x[t], w13, w2), ref[t], rtol=1e-11, atol=1e-14)
+
+
+def test_hidden_is_dense_swiglu_hidden():
+    """oracle.hidden gives silu(Wg x) * (Wu x) of each routed (token, slot),
+    against numpy matmuls, for the expert each slot names."""
+    wl = synth.workload("tiny").with_T(12)
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    w13 = synth.host_w13(wl)
+    a = oracle.hidden(oracle.cfg_for(wl), x, r["ids"], w13)
+    xf = f64(x)
+    for t in range(wl.T):
+        for k in range(wl.K):
+            w = f64(w13[r["ids"][t, k]])
+            g, u = w[:wl.I] @ xf[t], w[wl.I:] @ xf[t]
+            assert np.allclose(a[t, k], g * expit(g) * u, rtol=1e-11, atol=1e-14), (t, k)
 
 
 @pytest.mark.parametrize("renormalize", [True, False])
