@@ -14,6 +14,7 @@
 #include "beam_moe_oracle.h"
 
 #include <math.h>
+#include <pthread.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -254,10 +255,12 @@ int oracle_experts(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const in
 
 static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
 
-double oracle_e2m1_value(uint8_t code) {
+static double e2m1_value(uint8_t code) {
   double v = kE2M1[code & 7];
   return (code & 8) ? -v : v;
 }
+
+double oracle_e2m1_value(uint8_t code) { return e2m1_value(code); }
 
 double oracle_e4m3_value(uint8_t b) {
   int E = (b >> 3) & 15, f = b & 7;
@@ -319,10 +322,25 @@ int oracle_nvfp4_quantize(const float* v, int64_t K, float g, uint8_t* codes, ui
   return 0;
 }
 
-double oracle_nvfp4_value(const uint8_t* codes, const uint8_t* sf, int64_t i, double g) {
+/* Every E4M3 byte's value, filled once from oracle_e4m3_value so that the
+ * decoder below need not recompute it for each of the billions of elements a
+ * Beam-sized expert path reads; the values are oracle_e4m3_value's exactly. */
+static double g_e4m3[256];
+static pthread_once_t g_e4m3_once = PTHREAD_ONCE_INIT;
+static void fill_e4m3(void) {
+  for (int b = 0; b < 256; ++b) g_e4m3[b] = oracle_e4m3_value((uint8_t)b);
+}
+
+/* Element i of a packed row (the decoder every NVFP4 operand goes through). */
+static double nvfp4_value(const uint8_t* codes, const uint8_t* sf, int64_t i, double g) {
   uint8_t byte = codes[i / 2];
   uint8_t code = (i & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
-  return oracle_e2m1_value(code) * oracle_e4m3_value(sf[i / 16]) * g;
+  return e2m1_value(code) * g_e4m3[sf[i / 16]] * g;
+}
+
+double oracle_nvfp4_value(const uint8_t* codes, const uint8_t* sf, int64_t i, double g) {
+  pthread_once(&g_e4m3_once, fill_e4m3);
+  return nvfp4_value(codes, sf, i, g);
 }
 
 int oracle_experts_nvfp4(const oracle_cfg* cfg, int64_t T, const uint16_t* x, const int32_t* ids,
@@ -335,6 +353,7 @@ int oracle_experts_nvfp4(const oracle_cfg* cfg, int64_t T, const uint16_t* x, co
   if (!x || !ids || !weights || !w13_codes || !w13_sf || !w2_codes || !w2_sf || !out) return -1;
   const int H = cfg->hidden, I = cfg->inter, E = cfg->n_experts, K = cfg->top_k;
   if (H % 16 || I % 16) return -1;
+  pthread_once(&g_e4m3_once, fill_e4m3);
   int bad = 0;
 #pragma omp parallel
   {
@@ -358,7 +377,7 @@ int oracle_experts_nvfp4(const oracle_cfg* cfg, int64_t T, const uint16_t* x, co
           ot[h] = 0.0;
         }
         oracle_nvfp4_quantize(xf, H, g_x, xc, xs);
-        for (int h = 0; h < H; ++h) xd[h] = oracle_nvfp4_value(xc, xs, h, (double)g_x);
+        for (int h = 0; h < H; ++h) xd[h] = nvfp4_value(xc, xs, h, (double)g_x);
         for (int k = 0; k < K; ++k) {
           const int e = ids[t * K + k];
           if (e < 0 || e >= E || !w13_codes[e] || !w13_sf[e] || !w2_codes[e] || !w2_sf[e]) {
@@ -373,18 +392,18 @@ int oracle_experts_nvfp4(const oracle_cfg* cfg, int64_t T, const uint16_t* x, co
             const uint8_t* us = w13_sf[e] + (int64_t)(I + i) * (H / 16);
             double g = 0.0, u = 0.0;
             for (int h = 0; h < H; ++h) {
-              g += oracle_nvfp4_value(gc, gs, h, g_w13) * xd[h];
-              u += oracle_nvfp4_value(uc, us, h, g_w13) * xd[h];
+              g += nvfp4_value(gc, gs, h, g_w13) * xd[h];
+              u += nvfp4_value(uc, us, h, g_w13) * xd[h];
             }
             af[i] = (float)(g / (1.0 + exp(-g)) * u); /* silu(g) * u, then fp32 */
           }
           oracle_nvfp4_quantize(af, I, g_h, ac, as);
-          for (int i = 0; i < I; ++i) ad[i] = oracle_nvfp4_value(ac, as, i, (double)g_h);
+          for (int i = 0; i < I; ++i) ad[i] = nvfp4_value(ac, as, i, (double)g_h);
           for (int j = 0; j < H; ++j) {
             const uint8_t* dc = w2_codes[e] + (int64_t)j * (I / 2);
             const uint8_t* ds = w2_sf[e] + (int64_t)j * (I / 16);
             double acc = 0.0;
-            for (int i = 0; i < I; ++i) acc += oracle_nvfp4_value(dc, ds, i, g_w2) * ad[i];
+            for (int i = 0; i < I; ++i) acc += nvfp4_value(dc, ds, i, g_w2) * ad[i];
             ot[j] += weights[t * K + k] * acc;
           }
         }

@@ -75,7 +75,7 @@ MUTANTS = [
         ("swiglu_hidden(H, I, xd, w13[e], a + (t * K + k) * (int64_t)I);",
          "swiglu_hidden(H, I, xd, w13[e], a + t * (int64_t)I);")]),
     ("NVFP4 h not quantised", [
-        ("for (int i = 0; i < I; ++i) ad[i] = oracle_nvfp4_value(ac, as, i, (double)g_h);",
+        ("for (int i = 0; i < I; ++i) ad[i] = nvfp4_value(ac, as, i, (double)g_h);",
          "for (int i = 0; i < I; ++i) ad[i] = af[i];")]),
 ]
 
