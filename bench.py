@@ -1,19 +1,24 @@
 """Benchmark of the Beam MoE block forward on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all|decode|...]
                     [--impl ours|reference] [--no-cpu-baseline]
-                    [--format bf16|nvfp4] [--bias-mode 0|1] [--replay]
+                    [--format bf16|nvfp4] [--bias-mode 0|1] [--router-tc] [--replay]
 
 A step is one whole block forward (router GEMM, top-k, scan, permute, gate/up
 grouped GEMM, down grouped GEMM, combine) over one batch of T synthetic tokens
 with Beam's shapes: hidden 5120, 256 SwiGLU experts of intermediate 2560 in 8
-groups of 32, top-4 groups, top-8 experts, routed scale 2.5. The default
-workload is decode (T = 64), the configuration the throughput is quoted on.
-Weights and inputs are synthetic and seeded (bf16 experts N(0, 0.02), fp32
-router N(0, 1/sqrt(5120)), bf16 activations N(0, 1)); they are resident in HBM
-before timing starts. The L2 cache is flushed (256 MB write) before every
-timed step, outside the timed interval. Timing: CUDA events on the launching
-stream around each step, summed over K steps, max over ranks.
+groups of 32, top-4 groups, top-8 experts, routed scale 2.5. By default one
+run times all four Beam workloads on one set of expert weights: decode
+(T = 64), prefill (T = 4096), skewed routing (T = 16384) and the long prefill
+chunk (T = 65536, clustered inputs). The long chunk, the largest configuration
+that fits one GPU, is the line's headline (`value`, `roofline`, `e2e`,
+`cpu_baseline`); the other three sit under `workloads`, each with its own
+`roofline`, `e2e` and `clocks`. Weights and inputs are synthetic and seeded
+(bf16 experts N(0, 0.02), fp32 router N(0, 1/sqrt(5120)), bf16 activations
+N(0, 1)); they are resident in HBM before timing starts. The L2 cache is
+flushed (256 MB write) before every timed step, outside the timed interval.
+Timing: CUDA events on the launching stream around each step, summed over K
+steps, max over ranks.
 
 With N GPUs (torchrun, one process per GPU) every rank holds all experts and
 runs its own batch of T tokens: the block is data-parallel over tokens with
@@ -25,7 +30,7 @@ E2M1 codes, one E4M3 scale per 16 elements, an fp32 scale per tensor) on the
 block-scaled FP4 tensor cores; its tensor peak is 4x the measured bf16 peak.
 
 --impl reference times the fp64 CPU oracle (the reference arm of this
-repository) on a bounded sample of the same workload on the host cores.
+repository) on a bounded sample of the headline workload on the host cores.
 """
 import argparse
 import json
@@ -48,17 +53,13 @@ METRIC = "MoE-block tokens/s; achieved TFLOP/s or HBM GB/s as % of B200 roofline
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 STAGES = ("router_gemm", "router_topk", "scan", "permute", "gateup_gemm", "down_gemm", "combine")
-# router weight split, router GEMM, top-k, scan, permute, gate/up, down, combine;
-# replayed routes skip the first two and add one kernel that copies the routes in
-KERNELS_PER_STEP = 8
-KERNELS_PER_REPLAY_STEP = 6
 GEMM_SOURCES = ("sparse_moe_layer_beam_b200/csrc/grouped_gemm.cu",
                 "sparse_moe_layer_beam_b200/csrc/grouped_gemm.cuh",
                 "sparse_moe_layer_beam_b200/csrc/sm100.cuh")
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the gate/up
-# kernel per touched expert, from the ncu capture summarised in
-# profiles/grouped_gemm_decode_E32_T8.md; valid only for the decode workload and
-# only while the kernel sources hash to `sources_sha256`.
+# kernel per touched expert, from an ncu capture of the same kernel on a small
+# decode-like case; valid only for the decode workload and only while the
+# kernel sources hash to `sources_sha256` (any edit to them voids it).
 GATEUP_TRAFFIC = {"workload": "decode", "bytes_per_touched_expert": 52619897,
                   "sources_sha256": "d2654dc8e6ea4346cb90aa5c6d956b21c8ca1ae00fcb5da28860253f4dd80d0b"}
 
@@ -315,47 +316,50 @@ def rank_seed(rank):
     return synth.SEED + rank
 
 
-def run_ours(args, wl):
+class Experts:
+    """The expert weights every workload of one run shares (seed 0), on the
+    device: bf16 W13 / W2, or NVFP4 codes and scales."""
+
+    def __init__(self, wl, fmt, dev, st):
+        import torch
+
+        import sparse_moe_layer_beam_b200 as bm
+
+        self.nvfp4 = fmt == "nvfp4"
+        if self.nvfp4:
+            self.c13 = torch.empty(wl.w13_elems // 2, dtype=torch.uint8, device=dev)
+            self.s13 = torch.empty(wl.w13_elems // 16, dtype=torch.uint8, device=dev)
+            self.c2 = torch.empty(wl.w2_elems // 2, dtype=torch.uint8, device=dev)
+            self.s2 = torch.empty(wl.w2_elems // 16, dtype=torch.uint8, device=dev)
+            synth.dev_w13_nvfp4(wl, self.c13.data_ptr(), self.s13.data_ptr(), st)
+            synth.dev_w2_nvfp4(wl, self.c2.data_ptr(), self.s2.data_ptr(), st)
+            self.experts = bm.nvfp4_experts(self.c13, self.s13, self.c2, self.s2,
+                                            synth.NVFP4_WEIGHT_SCALE, synth.NVFP4_WEIGHT_SCALE,
+                                            synth.NVFP4_ACT_SCALE, synth.NVFP4_ACT_SCALE)
+            self.w13 = self.w2 = None
+        else:
+            self.w13 = torch.empty(wl.w13_elems, dtype=torch.int16, device=dev)
+            self.w2 = torch.empty(wl.w2_elems, dtype=torch.int16, device=dev)
+            synth.dev_w13(wl, self.w13.data_ptr(), st)
+            synth.dev_w2(wl, self.w2.data_ptr(), st)
+            self.experts = None
+        self.wr = torch.from_numpy(synth.host_router(wl)).to(dev)
+
+
+def measure(args, wl, ex, dev, stream, rank, world, local):
+    """Times W warm-up and K timed steps of one workload (device events on the
+    launching stream, L2 flushed before each step), then the same number of
+    end-to-end steps through the host-buffer entry point. Returns the
+    workload's part of the JSON line (max over ranks) and the routed counts."""
     import torch
     import torch.distributed as dist
 
     import sparse_moe_layer_beam_b200 as bm
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=dev)
-    stream = torch.cuda.current_stream()
     st = stream.cuda_stream
-
+    nvfp4 = ex.nvfp4
     cfg = bm.beam_cfg(wl.H, wl.I, wl.E, wl.G, wl.Gk, wl.K, wl.renormalize, args.bias_mode,
-                      wl.scale)
-    # all ranks hold the same experts (seed 0); each rank routes its own tokens
-    nvfp4 = args.format == "nvfp4"
-    if nvfp4:
-        c13 = torch.empty(wl.w13_elems // 2, dtype=torch.uint8, device=dev)
-        s13 = torch.empty(wl.w13_elems // 16, dtype=torch.uint8, device=dev)
-        c2 = torch.empty(wl.w2_elems // 2, dtype=torch.uint8, device=dev)
-        s2 = torch.empty(wl.w2_elems // 16, dtype=torch.uint8, device=dev)
-        synth.dev_w13_nvfp4(wl, c13.data_ptr(), s13.data_ptr(), st)
-        synth.dev_w2_nvfp4(wl, c2.data_ptr(), s2.data_ptr(), st)
-        experts = bm.nvfp4_experts(c13, s13, c2, s2, synth.NVFP4_WEIGHT_SCALE,
-                                   synth.NVFP4_WEIGHT_SCALE, synth.NVFP4_ACT_SCALE,
-                                   synth.NVFP4_ACT_SCALE)
-        w13 = w2 = None
-    else:
-        w13 = torch.empty(wl.w13_elems, dtype=torch.int16, device=dev)
-        w2 = torch.empty(wl.w2_elems, dtype=torch.int16, device=dev)
-        synth.dev_w13(wl, w13.data_ptr(), st)
-        synth.dev_w2(wl, w2.data_ptr(), st)
-    wr = torch.from_numpy(synth.host_router(wl)).to(dev)
+                      wl.scale, router_tc=args.router_tc)
     bias = synth.host_bias(wl)
     b = None if bias is None else torch.from_numpy(bias).to(dev)
     x = torch.empty((wl.T, wl.H), dtype=torch.int16, device=dev)
@@ -367,23 +371,24 @@ def run_ours(args, wl):
                      dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
+    lay = bm.beam_moe_workspace_layout(cfg, wl.T)
 
     ids = torch.empty((wl.T, wl.K), dtype=torch.int32, device=dev)
     wts = torch.empty((wl.T, wl.K), dtype=torch.float32, device=dev)
     if args.replay:  # record the routes once; the timed steps replay them
-        bm.beam_moe_forward(cfg, x, wr, b, w13, w2, out, ws, ids, wts, counts, stream=st)
+        bm.beam_moe_forward(cfg, x, ex.wr, b, ex.w13, ex.w2, out, ws, ids, wts, counts, stream=st)
 
     def step(trace=None):
         if nvfp4:
-            bm.beam_moe_forward_nvfp4(cfg, x, wr, b, experts, out, ws, expert_counts=counts,
+            bm.beam_moe_forward_nvfp4(cfg, x, ex.wr, b, ex.experts, out, ws, expert_counts=counts,
                                       stream=st, trace=trace)
         elif args.replay:
-            bm.beam_moe_forward_routed(cfg, x, ids, wts, w13, w2, out, ws, counts, stream=st)
+            bm.beam_moe_forward_routed(cfg, x, ids, wts, ex.w13, ex.w2, out, ws, counts, stream=st)
         elif trace is None:
-            bm.beam_moe_forward(cfg, x, wr, b, w13, w2, out, ws, expert_counts=counts,
+            bm.beam_moe_forward(cfg, x, ex.wr, b, ex.w13, ex.w2, out, ws, expert_counts=counts,
                                 stream=st)
         else:
-            bm.beam_moe_forward_traced(cfg, x, wr, b, w13, w2, out, ws, trace,
+            bm.beam_moe_forward_traced(cfg, x, ex.wr, b, ex.w13, ex.w2, out, ws, trace,
                                        expert_counts=counts, stream=st)
 
     for _ in range(args.warmup):
@@ -391,7 +396,7 @@ def run_ours(args, wl):
         step()
     flags = bm.beam_moe_check(ws, st)
     if flags:
-        raise SystemExit(f"device status flags {flags:#x} after warm-up")
+        raise SystemExit(f"{wl.name}: device status flags {flags:#x} after warm-up")
 
     trace = None if args.replay else bm.Trace(args.steps)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -413,9 +418,11 @@ def run_ours(args, wl):
     total_ms = sum(a.elapsed_time(c) for a, c in ev)
     stage_ms = (np.full((args.steps, len(STAGES)), np.nan) if trace is None
                 else np.array(trace.read()))  # [steps][stages]
+    if trace is not None:
+        trace.close()
     flags = bm.beam_moe_check(ws, st)
     if flags:
-        raise SystemExit(f"device status flags {flags:#x} in the timed region")
+        raise SystemExit(f"{wl.name}: device status flags {flags:#x} in the timed region")
 
     # End to end with host buffers: pinned x in, out back. The forward goes
     # through beam_moe_forward_host (chunked, copies overlapped with compute);
@@ -425,15 +432,18 @@ def run_ours(args, wl):
     out_host = torch.empty_like(out, device="cpu").pin_memory()
     ws_h = None
     if not args.replay:
+        del ws
         op_h = bm.OP_FORWARD_NVFP4_HOST if nvfp4 else bm.OP_FORWARD_HOST
         ws_h = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T, op_h), dtype=torch.uint8,
                            device=dev)
 
     def e2e_step():
         if nvfp4:
-            bm.beam_moe_forward_nvfp4_host(cfg, x_host, wr, b, experts, out_host, ws_h, stream=st)
+            bm.beam_moe_forward_nvfp4_host(cfg, x_host, ex.wr, b, ex.experts, out_host, ws_h,
+                                           stream=st)
         elif not args.replay:
-            bm.beam_moe_forward_host(cfg, x_host, wr, b, w13, w2, out_host, ws_h, stream=st)
+            bm.beam_moe_forward_host(cfg, x_host, ex.wr, b, ex.w13, ex.w2, out_host, ws_h,
+                                     stream=st)
         else:
             x.copy_(x_host, non_blocking=True)
             step()
@@ -453,13 +463,13 @@ def run_ours(args, wl):
     e2e_ms = sum(a.elapsed_time(c) for a, c in e2e_ev)
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
-
     ms_step = total_ms / args.steps
     tokens = wl.T * world
     value = tokens / (ms_step / 1000.0)
     e2e_value = tokens / (e2e_ms / args.steps / 1000.0)
 
-    alg = algorithmic(wl, counts.cpu().numpy(), args.format)
+    routed = counts.cpu().numpy()
+    alg = algorithmic(wl, routed, args.format)
     peaks, peak_kind = load_peaks()
     stage_mean = {n: float(stage_ms[:, i].mean()) for i, n in enumerate(STAGES)}
     gate_ms = float(stage_ms[:, 4].mean()) if trace is not None else float("nan")
@@ -467,16 +477,20 @@ def run_ours(args, wl):
                            nvfp4)
     # the recorded DRAM traffic belongs to the bf16 gate/up kernel only
     roof["traffic"] = None if nvfp4 else gateup_traffic(wl, alg["touched_experts"])
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4" if nvfp4 else "bf16",
-        "data": "synthetic",
+    # router GEMM (plus the weight split on tensor cores), top-k, scan,
+    # permute, gate/up, down, combine; replayed routes: the route copy, scan,
+    # permute, gate/up, down, combine
+    per_step = 6 if args.replay else (8 if lay.router_tc else 7)
+    part = {
+        "value": value, "ms_per_step": ms_step,
         "config": {"workload": describe(wl) + (" [routes replayed]" if args.replay else "")
                    + (" [NVFP4 experts and activations]" if nvfp4 else "")
-                   + (" [selection-only bias]" if args.bias_mode == 1 else ""),
+                   + (" [selection-only bias]" if args.bias_mode == 1 else "")
+                   + (" [router GEMM on tensor cores]" if lay.router_tc else ""),
                    "T": wl.T, "tokens_per_rank": wl.T,
                    "l2": "flushed before every timed step (256 MB write, outside the events)",
+                   "router": "tensor cores (exact bf16 split)" if lay.router_tc
+                   else "FP32 FMA on CUDA cores",
                    "parallelism": f"replicas x{world} (token data parallel, no exchange)"},
         "roofline": roof,
         "block": block,
@@ -486,19 +500,57 @@ def run_ours(args, wl):
                 "call": ("copies around beam_moe_forward_routed" if args.replay else
                          ("beam_moe_forward_nvfp4_host" if nvfp4 else "beam_moe_forward_host")
                          + f" ({host_chunking(wl.T, nvfp4)})")},
-        "gpu_launches": (KERNELS_PER_REPLAY_STEP if args.replay else KERNELS_PER_STEP)
-        * args.steps,
+        "gpu_launches": per_step * args.steps,
         "clocks": clk,
     }
+    return part
+
+
+# The default run times every Beam workload; the line's headline is the last
+# (the long prefill chunk, the largest configuration that fits one GPU).
+DEFAULT_WORKLOADS = ("decode", "prefill", "skewed", "long")
+
+
+def run_ours(args, wls):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    stream = torch.cuda.current_stream()
+    # all ranks hold the same experts (seed 0); each rank routes its own tokens
+    ex = Experts(wls[-1], args.format, dev, stream.cuda_stream)
+    parts = {}
+    for wl in wls:
+        parts[wl.name] = measure(args, wl, ex, dev, stream, rank, world, local)
+        torch.cuda.empty_cache()
+    head_wl = wls[-1]
+    head = parts.pop(head_wl.name)
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4" if ex.nvfp4 else "bf16", "data": "synthetic",
+    }
+    line.update({k: v for k, v in head.items() if k not in ("value", "ms_per_step")})
+    if parts:
+        line["workloads"] = parts
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sample = OracleSample(wl, oracle_sample_size(wl))
+        sample = OracleSample(head_wl, oracle_sample_size(head_wl))
         v, dt = sample.run()
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": sample.threads,
                                 "kind": "oracle", "sample": sample.desc, "seconds": dt}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if trace is not None:
-        trace.close()
     if world > 1:
         dist.destroy_process_group()
     return 0
@@ -509,13 +561,17 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="all", choices=["all"] + sorted(synth.WORKLOADS),
+                    help="all (default): decode, prefill, skewed and long, the last one the "
+                         "headline; or one workload")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--bias-mode", type=int, default=0, choices=[0, 1],
                     help="0: router bias on the logits; 1: on the choice scores only")
     ap.add_argument("--format", default="bf16", choices=["bf16", "nvfp4"],
                     help="expert weight / activation format of the timed forward")
+    ap.add_argument("--router-tc", action="store_true",
+                    help="opt in to the router GEMM on tensor cores (exact bf16 split)")
     ap.add_argument("--replay", action="store_true",
                     help="time the expert path with recorded routes (beam_moe_forward_routed)")
     ap.add_argument("--tokens", type=int, default=None,
@@ -527,15 +583,19 @@ def main():
         raise SystemExit("--warmup must be at least 3")
     if args.replay and args.format != "bf16":
         raise SystemExit("--replay times the bf16 routed entry point only")
-    wl = synth.workload(args.workload)
-    if args.tokens is not None:
-        wl = wl.with_T(args.tokens)
-    if args.experts is not None:
-        import dataclasses
-        wl = dataclasses.replace(wl, name=f"{wl.name} (E={args.experts})", E=args.experts)
+    names = DEFAULT_WORKLOADS if args.workload == "all" else (args.workload,)
+    wls = []
+    for name in names:
+        wl = synth.workload(name)
+        if args.tokens is not None:
+            wl = wl.with_T(args.tokens)
+        if args.experts is not None:
+            import dataclasses
+            wl = dataclasses.replace(wl, name=f"{wl.name} (E={args.experts})", E=args.experts)
+        wls.append(wl)
     if args.impl == "reference":
-        return run_reference(args, wl)
-    return run_ours(args, wl)
+        return run_reference(args, wls[-1])
+    return run_ours(args, wls)
 
 
 if __name__ == "__main__":

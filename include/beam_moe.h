@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-/* Block configuration. Beam: {5120, 2560, 256, 8, 4, 8, 1, 0, 2.5f}.
+/* Block configuration. Beam: {5120, 2560, 256, 8, 4, 8, 1, 0, 2.5f, 0}.
  * Supported: hidden and inter multiples of 128; n_experts <= 512 and a
  * multiple of n_group; group size (n_experts / n_group) >= 2; top_k <= 32 and
  * top_k <= topk_group * group size; see beam_moe_status for the codes. */
@@ -61,6 +61,15 @@ typedef struct beam_moe_cfg {
                           1: bias added to the scores for choosing only,
                              weights from the unbiased scores (DeepSeek-V3) */
   float routed_scale;  /* S: multiplies the combined output (2.5 in Beam)  */
+  int32_t router_tc;   /* 0 (default): the FP32 router GEMM is a chain of
+                          FP32 FMAs on CUDA cores. 1 (opt-in): the same
+                          contraction on tensor cores, each FP32 router
+                          weight split exactly into three bf16 parts whose
+                          products with the bf16 x are exact, summed by the
+                          tensor core's FP32 accumulator (its rounding of
+                          the sums is not an FMA chain's; about 6x faster
+                          for large batches). Needs hidden % 64 == 0,
+                          else the CUDA-core kernel runs.                  */
 } beam_moe_cfg;
 
 typedef enum beam_moe_status {
@@ -119,7 +128,9 @@ BEAM_MOE_API beam_moe_status beam_moe_route(const beam_moe_cfg* cfg, int64_t T, 
  *    BEAM_MOE_ERR_WORKSPACE_TOO_SMALL before anything is launched.
  *  - The first call on a device looks up the array's device address for that
  *    device (once, with that device current); make that first call before
- *    any stream capture on the device.
+ *    any stream capture on the device. The address is kept for the life of
+ *    the process, so a device reset (cudaDeviceReset, or a reset of the
+ *    primary context) after the first call is not supported.
  *  - Every call on a device shares the one array: calls that may overlap on
  *    the GPU (different streams, no ordering between them) race and must be
  *    serialized by the caller.
@@ -251,6 +262,44 @@ BEAM_MOE_API beam_moe_status beam_moe_nvfp4_quantize(int64_t rows, int64_t K, co
                                                      void* stream);
 
 /*
+ * Inspection of intermediates. beam_moe_forward_stages runs the stages of
+ * beam_moe_forward up to and including `last_stage` (0 router GEMM, 1 top-k
+ * and chunk counts, 2 scan, 3 permute, 4 gate/up grouped GEMM, 5 down grouped
+ * GEMM, 6 combine; the numbering of the stage trace below) and leaves every
+ * intermediate in the workspace; with last_stage = 6 it is beam_moe_forward
+ * without the optional route outputs. out may be NULL unless last_stage is 6.
+ * beam_moe_workspace_layout reports where the intermediates sit for T tokens
+ * on the current device (byte offsets from the start of ws):
+ *   counts  [E] int32          rows routed to each expert
+ *   offsets [E+1] int32        first permuted row of each expert
+ *   ids, w  [T][K] int32/fp32  routes and combine weights (S included)
+ *   pos     [T][K] int32       permuted row of each (token, slot): the rows of
+ *                              an expert are contiguous from offsets[e], in
+ *                              ascending token order
+ *   xp      [T*K][H] bf16      permuted token rows (valid after stage 3 and
+ *                              until stage 5 overwrites them with y)
+ *   h       [T*K][I] bf16      silu(g) * u of each permuted row (after stage 4)
+ *   y       [T*K][H] fp32      down projection of each permuted row (after
+ *                              stage 5; the same bytes as xp)
+ * op must be BEAM_MOE_OP_ROUTE (only the routing arrays are meaningful) or
+ * BEAM_MOE_OP_FORWARD. These calls exist for tests and debugging.
+ */
+typedef struct beam_moe_ws_layout {
+  int64_t counts, offsets, ids, w, pos, xp, h, y; /* byte offsets in ws         */
+  int32_t router_splits; /* slices of H whose FP32 partial logits are added  */
+  int32_t router_tc;     /* 1: the router GEMM runs on tensor cores           */
+  int32_t pair_gateup;   /* 1: gate/up grouped GEMM on CTA pairs              */
+  int32_t pair_down;     /* 1: down grouped GEMM on CTA pairs                 */
+} beam_moe_ws_layout;
+BEAM_MOE_API beam_moe_status beam_moe_workspace_layout(const beam_moe_cfg* cfg, int64_t T,
+                                                       beam_moe_op op,
+                                                       beam_moe_ws_layout* layout);
+BEAM_MOE_API beam_moe_status beam_moe_forward_stages(
+    const beam_moe_cfg* cfg, int64_t T, const uint16_t* x, const float* w_router,
+    const float* bias, const uint16_t* w13, const uint16_t* w2, uint16_t* out,
+    int32_t last_stage, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Stage timing. A trace records CUDA events around each stage of the calls
  * it is passed to: slot i of stage s is the time of that stage in the i-th
  * traced call since the last reset. Stages: 0 router GEMM, 1 top-k and
@@ -358,7 +407,10 @@ BEAM_MOE_API beam_moe_status beam_moe_ep_combine(const beam_moe_cfg* cfg,
  * 0x2 MMA issuer, 0x4 epilogue gave up a bounded wait; 0x100 an expert id
  * outside [0, E) reached the dispatch; 0x200 beam_moe_selftest_wait's wait ran
  * out; 0x400 a received row's return address named no rank or slot (the row
- * is not stored; only inconsistent recv_counts lead there). Returns
+ * is not stored; only inconsistent recv_counts lead there); 0x800 a
+ * dispatched row's place in its owner's receive buffer fell outside
+ * [0, recv_cap) (the row is not stored; send_base from another step's plan
+ * leads there). Returns
  * BEAM_MOE_ERR_DEVICE_TIMEOUT
  * if any bit was set, BEAM_MOE_ERR_CUDA if the stream reports an error.
  */

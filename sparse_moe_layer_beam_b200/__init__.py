@@ -23,6 +23,7 @@ __all__ = ["BeamMoeCfg", "BeamMoeError", "Trace", "OP_ROUTE", "OP_FORWARD", "N_S
            "beam_moe_ep_route", "beam_moe_ep_plan", "beam_moe_ep_dispatch", "beam_moe_ep_experts",
            "beam_moe_ep_combine", "beam_moe_selftest_wait",
            "beam_moe_forward", "beam_moe_forward_routed", "beam_moe_forward_traced",
+           "beam_moe_forward_stages", "beam_moe_workspace_layout", "BeamMoeWsLayout",
            "beam_moe_check"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -44,7 +45,16 @@ class BeamMoeCfg(ctypes.Structure):
                 ("n_experts", ctypes.c_int32), ("n_group", ctypes.c_int32),
                 ("topk_group", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("renormalize", ctypes.c_int32), ("bias_mode", ctypes.c_int32),
-                ("routed_scale", ctypes.c_float)]
+                ("routed_scale", ctypes.c_float), ("router_tc", ctypes.c_int32)]
+
+
+class BeamMoeWsLayout(ctypes.Structure):
+    """Byte offsets of the intermediates inside a forward workspace."""
+    _fields_ = [("counts", ctypes.c_int64), ("offsets", ctypes.c_int64), ("ids", ctypes.c_int64),
+                ("w", ctypes.c_int64), ("pos", ctypes.c_int64), ("xp", ctypes.c_int64),
+                ("h", ctypes.c_int64), ("y", ctypes.c_int64), ("router_splits", ctypes.c_int32),
+                ("router_tc", ctypes.c_int32), ("pair_gateup", ctypes.c_int32),
+                ("pair_down", ctypes.c_int32)]
 
 
 class BeamMoeNvfp4Experts(ctypes.Structure):
@@ -78,6 +88,10 @@ _SIGS = {
     "beam_moe_route_noalloc": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P],
     "beam_moe_forward": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                          ctypes.c_size_t, _P],
+    "beam_moe_forward_stages": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, ctypes.c_int32,
+                                _P, ctypes.c_size_t, _P],
+    "beam_moe_workspace_layout": [_CFG, ctypes.c_int64, ctypes.c_int,
+                                  ctypes.POINTER(BeamMoeWsLayout)],
     "beam_moe_forward_routed": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P,
                                 ctypes.c_size_t, _P],
     "beam_moe_forward_traced": [_CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -126,9 +140,13 @@ def lib():
     return _lib
 
 
-def beam_cfg(H=5120, I=2560, E=256, G=8, Gk=4, K=8, renormalize=True, bias_mode=0, scale=2.5):
-    """Configuration struct; the defaults are the Beam block."""
-    return BeamMoeCfg(H, I, E, G, Gk, K, 1 if renormalize else 0, bias_mode, scale)
+def beam_cfg(H=5120, I=2560, E=256, G=8, Gk=4, K=8, renormalize=True, bias_mode=0, scale=2.5,
+             router_tc=False):
+    """Configuration struct; the defaults are the Beam block. router_tc opts in
+    to the router GEMM on tensor cores (exact three-way bf16 split of the FP32
+    weights); the default is FP32 FMAs on CUDA cores."""
+    return BeamMoeCfg(H, I, E, G, Gk, K, 1 if renormalize else 0, bias_mode, scale,
+                      1 if router_tc else 0)
 
 
 def _check(status, where):
@@ -191,6 +209,24 @@ def beam_moe_forward_traced(cfg, x, w_router, bias, w13, w2, out, ws, trace, top
                                          _ptr(ws), ws.numel() * ws.element_size(),
                                          _stream(stream), trace.handle),
            "beam_moe_forward_traced")
+
+
+def beam_moe_forward_stages(cfg, x, w_router, bias, w13, w2, out, last_stage, ws, stream=None):
+    """The forward's stages 0..last_stage (0 router GEMM ... 6 combine), leaving
+    the intermediates in ws (see beam_moe_workspace_layout)."""
+    T = x.shape[0]
+    _check(lib().beam_moe_forward_stages(ctypes.byref(cfg), T, _ptr(x), _ptr(w_router),
+                                         _ptr(bias), _ptr(w13), _ptr(w2), _ptr(out), last_stage,
+                                         _ptr(ws), ws.numel() * ws.element_size(),
+                                         _stream(stream)), "beam_moe_forward_stages")
+
+
+def beam_moe_workspace_layout(cfg, T, op=OP_FORWARD):
+    """BeamMoeWsLayout of a workspace for T tokens on the current device."""
+    out = BeamMoeWsLayout()
+    _check(lib().beam_moe_workspace_layout(ctypes.byref(cfg), T, op, ctypes.byref(out)),
+           "beam_moe_workspace_layout")
+    return out
 
 
 def beam_moe_forward_routed(cfg, x, topk_ids, topk_w, w13, w2, out, ws, expert_counts=None,

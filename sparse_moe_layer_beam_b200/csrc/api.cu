@@ -19,17 +19,15 @@ extern "C" BEAM_MOE_API beam_moe_status beam_moe_workspace_size(const beam_moe_c
 namespace beam {
 
 int device_sm_count() {
-  static int cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        sms <= 0)
-      sms = 148;
-    cached[dev] = sms;
-  }
-  return cached[dev];
+  static PerDevice cached;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  const cudaError_t err = cached.get(dev, &sms, [dev](int* v) {
+    if (cudaDeviceGetAttribute(v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || *v <= 0)
+      *v = 148;
+    return cudaSuccess;
+  });
+  return err == cudaSuccess ? sms : 148;
 }
 
 int router_split_k(int64_t T, int H, int E, int sms);
@@ -46,14 +44,14 @@ static int pick_bn(int64_t T, int K, int E) {
   return 256;
 }
 
-Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool tc_router) {
+Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool allow_tc) {
   Layout L;
   memset(&L, 0, sizeof(L));
   const int E = c.n_experts, K = c.top_k, H = c.hidden, I = c.inter;
   L.T = T;
   L.A = T * K;
   L.nchunks = (int)((T + kChunk - 1) / kChunk);
-  L.router_tc = (tc_router && router_tc_supported(c)) ? 1 : 0;
+  L.router_tc = (allow_tc && c.router_tc == 1 && router_tc_supported(c)) ? 1 : 0;
   if (L.router_tc) {
     const int nkb = H / 64;
     L.router_kper = router_tc_kper(T, H, E, sms);
@@ -178,6 +176,7 @@ static beam_moe_status check_cfg(const beam_moe_cfg* c) {
     return BEAM_MOE_ERR_INVALID_ARG;
   if (c->renormalize != 0 && c->renormalize != 1) return BEAM_MOE_ERR_INVALID_ARG;
   if (c->bias_mode != 0 && c->bias_mode != 1) return BEAM_MOE_ERR_INVALID_ARG;
+  if (c->router_tc != 0 && c->router_tc != 1) return BEAM_MOE_ERR_INVALID_ARG;
   if (!isfinite(c->routed_scale)) return BEAM_MOE_ERR_INVALID_ARG;
   if (c->n_experts % c->n_group != 0 || c->topk_group > c->n_group) return BEAM_MOE_ERR_INVALID_ARG;
   const int gs = c->n_experts / c->n_group;
@@ -278,45 +277,56 @@ beam_moe_status plan(const beam_moe_cfg* cfg, int64_t T, Layout* L) {
   return BEAM_MOE_OK;
 }
 
+// Stages 2..last of a forward (scan, permute, gate/up, down, combine).
 beam_moe_status expert_path(const beam_moe_cfg* cfg, const Layout& L, const uint16_t* x,
                             const uint16_t* w13, const uint16_t* w2, uint16_t* out,
-                            int32_t* counts_out, char* ws, cudaStream_t st, Recorder& rec) {
+                            int32_t* counts_out, char* ws, cudaStream_t st, Recorder& rec,
+                            int last = 6) {
   BEAM_CUDA(beam::launch_scan(*cfg, L, ws, counts_out, st));
   BEAM_CUDA(rec.mark(3));
+  if (last < 3) return BEAM_MOE_OK;
   BEAM_CUDA(beam::launch_permute(*cfg, L, x, ws, st));
   BEAM_CUDA(rec.mark(4));
+  if (last < 4) return BEAM_MOE_OK;
   BEAM_CUDA(L.pair_gateup ? beam::launch_gateup_pair(*cfg, L, w13, ws, st)
                    : beam::launch_gateup(*cfg, L, w13, ws, st));
   BEAM_CUDA(rec.mark(5));
+  if (last < 5) return BEAM_MOE_OK;
   BEAM_CUDA(L.pair_down ? beam::launch_down_pair(*cfg, L, w2, ws, st)
                    : beam::launch_down(*cfg, L, w2, ws, st));
   BEAM_CUDA(rec.mark(6));
+  if (last < 6) return BEAM_MOE_OK;
   BEAM_CUDA(beam::launch_combine(*cfg, L, out, ws, st));
   BEAM_CUDA(rec.mark(7));
   return BEAM_MOE_OK;
 }
 
+// A forward through stage `last` (6: the whole block).
 beam_moe_status forward_impl(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
                              const float* w_router, const float* bias, const uint16_t* w13,
                              const uint16_t* w2, uint16_t* out, int32_t* topk_ids, float* topk_w,
                              int32_t* expert_counts, void* ws, size_t ws_bytes, void* stream,
-                             beam_moe_trace* trace) {
+                             beam_moe_trace* trace, int last = 6) {
   BEAM_TRY(common_checks(cfg, T, ws, ws_bytes, BEAM_MOE_OP_FORWARD));
+  if (last < 0 || last > 6) return BEAM_MOE_ERR_INVALID_ARG;
   if (T == 0) return BEAM_MOE_OK;
-  BEAM_TRY(check_ptrs({x, w_router, w13, w2, out}, {bias, topk_ids, topk_w, expert_counts}));
+  BEAM_TRY(check_ptrs({x, w_router, w13, w2}, {bias, topk_ids, topk_w, expert_counts, out}));
+  if (last == 6 && !out) return BEAM_MOE_ERR_INVALID_ARG;
   Layout L;
   BEAM_TRY(plan(cfg, T, &L));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
-  Recorder rec(trace, st);
+  Recorder rec(last == 6 ? trace : nullptr, st);
   BEAM_CUDA(cudaMemsetAsync(w + L.status, 0, 256, st));
   BEAM_CUDA(rec.mark(0));
   BEAM_CUDA(beam::launch_router_logits(*cfg, L, x, w_router, w, st));
   BEAM_CUDA(rec.mark(1));
-  BEAM_CUDA(beam::launch_router_topk(*cfg, L, bias, w, st));
-  BEAM_CUDA(rec.mark(2));
-  BEAM_TRY(expert_path(cfg, L, x, w13, w2, out, expert_counts, w, st, rec));
-  BEAM_CUDA(beam::launch_copy_routes(*cfg, L, topk_ids, topk_w, w, st));
+  if (last >= 1) {
+    BEAM_CUDA(beam::launch_router_topk(*cfg, L, bias, w, st));
+    BEAM_CUDA(rec.mark(2));
+  }
+  if (last >= 2) BEAM_TRY(expert_path(cfg, L, x, w13, w2, out, expert_counts, w, st, rec, last));
+  if (last >= 1) BEAM_CUDA(beam::launch_copy_routes(*cfg, L, topk_ids, topk_w, w, st));
   rec.done();
   return BEAM_MOE_OK;
 }
@@ -616,6 +626,38 @@ beam_moe_status beam_moe_forward(const beam_moe_cfg* cfg, int64_t T, const uint1
                       ws, ws_bytes, stream, nullptr);
 }
 
+beam_moe_status beam_moe_forward_stages(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
+                                        const float* w_router, const float* bias,
+                                        const uint16_t* w13, const uint16_t* w2, uint16_t* out,
+                                        int32_t last_stage, void* ws, size_t ws_bytes,
+                                        void* stream) {
+  return forward_impl(cfg, T, x, w_router, bias, w13, w2, out, nullptr, nullptr, nullptr, ws,
+                      ws_bytes, stream, nullptr, last_stage);
+}
+
+beam_moe_status beam_moe_workspace_layout(const beam_moe_cfg* cfg, int64_t T, beam_moe_op op,
+                                          beam_moe_ws_layout* out) {
+  BEAM_TRY(check_cfg(cfg));
+  BEAM_TRY(check_T(cfg, T));
+  if (!out || (op != BEAM_MOE_OP_ROUTE && op != BEAM_MOE_OP_FORWARD))
+    return BEAM_MOE_ERR_INVALID_ARG;
+  Layout L;
+  BEAM_TRY(plan(cfg, T, &L));
+  out->counts = (int64_t)L.counts;
+  out->offsets = (int64_t)L.offsets;
+  out->ids = (int64_t)L.ids;
+  out->w = (int64_t)L.w;
+  out->pos = (int64_t)L.pos;
+  out->xp = (int64_t)L.xp;
+  out->h = (int64_t)L.h;
+  out->y = (int64_t)L.xp;
+  out->router_splits = L.split_k;
+  out->router_tc = L.router_tc;
+  out->pair_gateup = L.pair_gateup;
+  out->pair_down = L.pair_down;
+  return BEAM_MOE_OK;
+}
+
 beam_moe_status beam_moe_forward_traced(const beam_moe_cfg* cfg, int64_t T, const uint16_t* x,
                                         const float* w_router, const float* bias,
                                         const uint16_t* w13, const uint16_t* w2, uint16_t* out,
@@ -728,7 +770,7 @@ Layout ep_routing(const beam_moe_cfg& c, int64_t T, int sms, size_t base) {
 // 4096, then the last T of every 128-token block (both routers' token tiles
 // are whole 128-token blocks there, so within one block the split is fixed
 // and the size grows with T).
-size_t ep_route_bytes(const beam_moe_cfg& c, int64_t t_max) {
+size_t ep_route_bytes_scan(const beam_moe_cfg& c, int64_t t_max) {
   size_t best = 0;
   for (int64_t t = 1; t <= t_max; t = (t < 4096 ? t + 1 : (t + 128) / 128 * 128)) {
     const Layout L = beam::make_layout(c, t, 1024);
@@ -740,6 +782,28 @@ size_t ep_route_bytes(const beam_moe_cfg& c, int64_t t_max) {
     }
   }
   return best;
+}
+
+// ep_route_bytes_scan's result, remembered per (configuration, t_max): every
+// phase of an expert-parallel step checks its workspace size, and the scan
+// walks thousands of layouts.
+size_t ep_route_bytes(const beam_moe_cfg& c, int64_t t_max) {
+  struct Entry {
+    beam_moe_cfg cfg;
+    int64_t t_max;
+    size_t bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> seen;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : seen)
+      if (e.t_max == t_max && memcmp(&e.cfg, &c, sizeof(c)) == 0) return e.bytes;
+  }
+  const size_t bytes = ep_route_bytes_scan(c, t_max);
+  std::lock_guard<std::mutex> lock(mu);
+  if (seen.size() < 64) seen.push_back({c, t_max, bytes});
+  return bytes;
 }
 
 beam_moe_status ep_ws_checks(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep, void* ws,

@@ -64,14 +64,17 @@ EpLayout make_ep_layout(const beam_moe_cfg& c, const beam_moe_ep_cfg& g) {
 namespace {
 
 // One CTA per local token: the K return addresses and combine positions,
-// then the token's row copied to each owner's receive buffer.
+// then the token's row copied to each owner's receive buffer. A row whose
+// place in the owner's buffer falls outside [0, recv_cap) (send_base from
+// another step's plan, for instance) is never stored: it is dropped, its
+// combine position is -1 and status bit kFlagBadDispatch is set.
 __global__ void __launch_bounds__(128) ep_dispatch_kernel(
     const uint16_t* __restrict__ x, int H, int K, int E, int El, int rank,
     const int32_t* __restrict__ ids, const int32_t* __restrict__ chunk_base,
     const uint32_t* __restrict__ chunk_mask, const int32_t* __restrict__ offsets,
     const int32_t* __restrict__ send_base, int32_t* __restrict__ pos,
     const __grid_constant__ Peers peers,
-    size_t recv_off, size_t src_off) {
+    size_t recv_off, size_t src_off, int64_t recv_cap, unsigned* status) {
   __shared__ uint16_t* s_dst[32];
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
@@ -85,11 +88,17 @@ __global__ void __launch_bounds__(128) ep_dispatch_kernel(
       int r = 0;
       for (int wd = 0; wd < (tl >> 5); ++wd) r += __popc(m[wd]);
       r += __popc(m[tl >> 5] & ((1u << (tl & 31)) - 1u));
-      const int row = send_base[e] + (chunk_base[(size_t)c * E + e] + r - offsets[e]);
-      char* peer = peers.ws[e / El];
-      dst = reinterpret_cast<uint16_t*>(peer + recv_off) + (size_t)row * H;
-      reinterpret_cast<int32_t*>(peer + src_off)[row] = (rank << kSlotBits) | (int)slot;
-      pos[slot] = (int)slot;
+      const int64_t row =
+          (int64_t)send_base[e] + (chunk_base[(size_t)c * E + e] + r - offsets[e]);
+      if (row >= 0 && row < recv_cap) {
+        char* peer = peers.ws[e / El];
+        dst = reinterpret_cast<uint16_t*>(peer + recv_off) + (size_t)row * H;
+        reinterpret_cast<int32_t*>(peer + src_off)[row] = (rank << kSlotBits) | (int)slot;
+        pos[slot] = (int)slot;
+      } else {
+        atomicOr(status, kFlagBadDispatch);
+        pos[slot] = -1;
+      }
     } else {
       pos[slot] = -1;
     }
@@ -141,7 +150,8 @@ cudaError_t launch_ep_dispatch(const beam_moe_cfg& c, const beam_moe_ep_cfg& g,
       reinterpret_cast<const int32_t*>(wr + L.ids), reinterpret_cast<const int32_t*>(wr + L.chunk_cnt),
       reinterpret_cast<const uint32_t*>(wr + L.chunk_mask),
       reinterpret_cast<const int32_t*>(wr + L.offsets), send_base,
-      reinterpret_cast<int32_t*>(wr + L.pos), peers, P.recv, P.src);
+      reinterpret_cast<int32_t*>(wr + L.pos), peers, P.recv, P.src, g.recv_cap,
+      reinterpret_cast<unsigned*>(wr + P.status));
   return cudaGetLastError();
 }
 

@@ -258,16 +258,13 @@ template <bool GATEUP, int BN>
 cudaError_t run(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p,
                 cudaStream_t st) {
   using C = Cfg<GATEUP, BN>;
-  static int configured_device = -1;  // attribute set once per process and device
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+  static PerDevice configured;  // the shared-memory attribute, once per device
+  int unused = 0;
+  cudaError_t err = per_device(configured, &unused, [](int*) {
+    return cudaFuncSetAttribute(grouped_gemm_kernel<GATEUP, BN>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  });
   if (err != cudaSuccess) return err;
-  if (configured_device != dev) {
-    err = cudaFuncSetAttribute(grouped_gemm_kernel<GATEUP, BN>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (err != cudaSuccess) return err;
-    configured_device = dev;
-  }
   grouped_gemm_kernel<GATEUP, BN><<<device_sm_count(), kThreads, C::kSmemBytes, st>>>(tw, tx, p);
   return cudaGetLastError();
 }

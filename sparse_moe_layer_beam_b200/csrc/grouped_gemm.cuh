@@ -46,12 +46,19 @@ __device__ __forceinline__ void decode_tile(int tile, const GemmParams& p, int& 
   nb = local - mb * nblk;
 }
 
-// silu(g) u in FP32, with silu(g) = g sigmoid(g) = (g/2)(1 + tanh(g/2)): one
-// hardware tanh (relative error about 2^-11) instead of an exponential and a
-// reciprocal. The error, at most about 2^-11 |g|/2 in silu, stays below the
-// bf16 (or E2M1) rounding that h gets next, and the cheaper epilogue runs
-// the power-capped GEMMs a little faster.
+// silu(g) u in FP32 for the bf16 path: silu(g) = g / (1 + e^-g) with the
+// hardware exponential and an approximate FP32 division, both within a few
+// FP32 ulps, so h = silu(g) u is FP32-accurate before its one bf16 rounding
+// (the SwiGLU product is FP32 in "Welcome Beam", section "Residual Stream").
+// For g below about -88, e^-g overflows to +inf and the quotient is -0.
 __device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
+// silu(g) u for the NVFP4 path, where h is quantised to E2M1 (4 bits) next:
+// silu(g) = (g/2)(1 + tanh(g/2)) with one hardware tanh (relative error about
+// 2^-11), far below the E2M1 step, instead of an exponential and a division.
+__device__ __forceinline__ float silu_mul_fast(float g, float u) {
   const float hg = 0.5f * g;
   float t;
   asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hg));

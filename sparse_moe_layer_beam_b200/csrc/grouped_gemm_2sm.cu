@@ -321,11 +321,7 @@ cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const CUtenso
   // Per device: the shared-memory attribute and the number of CTA pairs that
   // can be resident at once (a pair needs two SMs of one GPC). The grid is
   // exactly that many pairs, so no pair waits for another to finish.
-  static int configured_device = -1;
-  static int resident_pairs = 0;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
+  static PerDevice pairs;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -337,18 +333,21 @@ cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const CUtenso
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (configured_device != dev) {
-    err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATEUP, EPRET>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::kSmemBytes);
-    if (err != cudaSuccess) return err;
-    cfg.gridDim = dim3((unsigned)(device_sm_count() & ~1));
+  int resident_pairs = 0;
+  cudaError_t err = per_device(pairs, &resident_pairs, [&cfg](int* v) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATEUP, EPRET>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t probe = cfg;
+    probe.gridDim = dim3((unsigned)(device_sm_count() & ~1));
     int clusters = 0;
-    err = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<GATEUP, EPRET>, &cfg);
-    if (err != cudaSuccess) return err;
+    e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<GATEUP, EPRET>, &probe);
+    if (e != cudaSuccess) return e;
     if (clusters < 1) return cudaErrorInvalidConfiguration;
-    resident_pairs = clusters < device_sm_count() / 2 ? clusters : device_sm_count() / 2;
-    configured_device = dev;
-  }
+    *v = clusters < device_sm_count() / 2 ? clusters : device_sm_count() / 2;
+    return cudaSuccess;
+  });
+  if (err != cudaSuccess) return err;
   cfg.gridDim = dim3((unsigned)(2 * resident_pairs));
   return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATEUP, EPRET>, tw, tx, tx64, p, ret);
 }

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "beam_moe.h"
 
 namespace beam {
@@ -27,6 +29,44 @@ constexpr uint32_t kFlagEpilogue = 0x4;
 constexpr uint32_t kFlagBadExpert = 0x100;
 constexpr uint32_t kFlagSelftest = 0x200;  // beam_moe_selftest_wait's wait ran out
 constexpr uint32_t kFlagBadReturn = 0x400; // a received row's return address out of range
+constexpr uint32_t kFlagBadDispatch = 0x800; // a dispatched row would land outside recv_cap
+
+// A value set up once per device (a kernel's shared-memory attribute, the
+// number of CTA pairs that can be resident), for host code that launches on
+// several devices from several threads. get() runs setup(&v) under the lock
+// the first time it is asked for `dev`; a failed set-up is retried next time.
+class PerDevice {
+ public:
+  static constexpr int kMaxDevices = 64;
+  template <class F>
+  cudaError_t get(int dev, int* out, F&& setup) {
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (!done_[dev]) {
+      int v = 0;
+      const cudaError_t err = setup(&v);
+      if (err != cudaSuccess) return err;
+      val_[dev] = v;
+      done_[dev] = true;
+    }
+    *out = val_[dev];
+    return cudaSuccess;
+  }
+
+ private:
+  std::mutex mu_;
+  int val_[kMaxDevices] = {};
+  bool done_[kMaxDevices] = {};
+};
+
+// The current device's PerDevice value (cudaGetDevice, then get()).
+template <class F>
+cudaError_t per_device(PerDevice& pd, int* out, F&& setup) {
+  int dev = 0;
+  const cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  return pd.get(dev, out, setup);
+}
 
 // Byte offsets of every scratch array inside the caller's workspace.
 struct Layout {
@@ -56,8 +96,10 @@ struct Layout {
   size_t total;     // bytes needed by the forward op
 };
 
-// tc_router = false keeps the router on CUDA cores (no weight planes needed).
-Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool tc_router = true);
+// The router GEMM runs on tensor cores only when the configuration asks for
+// it (c.router_tc) and allow_tc is set; allow_tc = false keeps it on CUDA
+// cores whatever the configuration says (no weight planes needed).
+Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool allow_tc = true);
 
 // NVFP4 path: the routing layout (token tiles of 128 rows, expert segments
 // padded to them) plus quantised activations and their scales.

@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              hb[j] = __float_as_uint(gg::silu_mul(__uint_as_float(g[j]) * p.acc_scale,
+              hb[j] = __float_as_uint(gg::silu_mul_fast(__uint_as_float(g[j]) * p.acc_scale,
                                                    __uint_as_float(u[j]) * p.acc_scale));
             tmem_st16(tp + 16 * c, hb);
           }
@@ -553,16 +553,13 @@ template <bool GATEUP>
 cudaError_t run4(const CUtensorMap& tw, const CUtensorMap& tx, const Fp4Params& p,
                  cudaStream_t st) {
   using C = Cfg4<GATEUP>;
-  static int configured_device = -1;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+  static PerDevice configured;  // the shared-memory attribute, once per device
+  int unused = 0;
+  cudaError_t err = per_device(configured, &unused, [](int*) {
+    return cudaFuncSetAttribute(grouped_gemm_nvfp4_kernel<GATEUP>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  });
   if (err != cudaSuccess) return err;
-  if (configured_device != dev) {
-    err = cudaFuncSetAttribute(grouped_gemm_nvfp4_kernel<GATEUP>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (err != cudaSuccess) return err;
-    configured_device = dev;
-  }
   grouped_gemm_nvfp4_kernel<GATEUP><<<device_sm_count(), C::kThreads, C::kSmemBytes, st>>>(tw, tx, p);
   return cudaGetLastError();
 }

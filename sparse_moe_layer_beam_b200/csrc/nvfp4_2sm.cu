@@ -367,11 +367,7 @@ cudaError_t launch_down_nvfp4_pair(const beam_moe_cfg& c, const Fp4Layout& F,
 
   // Per device: the shared-memory attribute and the number of CTA pairs that
   // can be resident at once. The grid is exactly that many pairs.
-  static int configured_device = -1;
-  static int resident_pairs = 0;
-  int dev = 0;
-  err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
+  static PerDevice pairs;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -383,18 +379,21 @@ cudaError_t launch_down_nvfp4_pair(const beam_moe_cfg& c, const Fp4Layout& F,
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (configured_device != dev) {
-    err = cudaFuncSetAttribute(down_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               P4Cfg::kSmemBytes);
-    if (err != cudaSuccess) return err;
-    cfg.gridDim = dim3((unsigned)(device_sm_count() & ~1));
+  int resident_pairs = 0;
+  err = per_device(pairs, &resident_pairs, [&cfg](int* v) {
+    cudaError_t e = cudaFuncSetAttribute(down_nvfp4_pair_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, P4Cfg::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t probe = cfg;
+    probe.gridDim = dim3((unsigned)(device_sm_count() & ~1));
     int clusters = 0;
-    err = cudaOccupancyMaxActiveClusters(&clusters, down_nvfp4_pair_kernel, &cfg);
-    if (err != cudaSuccess) return err;
+    e = cudaOccupancyMaxActiveClusters(&clusters, down_nvfp4_pair_kernel, &probe);
+    if (e != cudaSuccess) return e;
     if (clusters < 1) return cudaErrorInvalidConfiguration;
-    resident_pairs = clusters < device_sm_count() / 2 ? clusters : device_sm_count() / 2;
-    configured_device = dev;
-  }
+    *v = clusters < device_sm_count() / 2 ? clusters : device_sm_count() / 2;
+    return cudaSuccess;
+  });
+  if (err != cudaSuccess) return err;
   cfg.gridDim = dim3((unsigned)(2 * resident_pairs));
   return cudaLaunchKernelEx(&cfg, down_nvfp4_pair_kernel, tw, tx, p);
 }

@@ -254,16 +254,13 @@ template <int BN>
 cudaError_t run_router_tc(const CUtensorMap& tw, const CUtensorMap& tx, const RouterTcParams& p,
                           cudaStream_t st) {
   using C = RCfg<BN>;
-  static int configured_device = -1;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+  static PerDevice configured;  // the shared-memory attribute, once per device
+  int unused = 0;
+  cudaError_t err = per_device(configured, &unused, [](int*) {
+    return cudaFuncSetAttribute(router_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::kSmemBytes);
+  });
   if (err != cudaSuccess) return err;
-  if (configured_device != dev) {
-    err = cudaFuncSetAttribute(router_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               C::kSmemBytes);
-    if (err != cudaSuccess) return err;
-    configured_device = dev;
-  }
   const int total = p.n_split * p.n_nt * p.n_mb;
   const int grid = total < device_sm_count() ? total : device_sm_count();
   router_tc_kernel<BN><<<grid, kRThreads, C::kSmemBytes, st>>>(tw, tx, p);

@@ -1,7 +1,12 @@
 """GPU-side helpers for parity tests and the smoke check: device buffers filled
 by the synthetic generator, a forward call through the C ABI, and the oracle
 comparison on sampled tokens. Expected values come only from oracle/."""
+import collections
+import concurrent.futures
+import os
+
 import numpy as np
+import psutil
 import torch
 
 import oracle
@@ -86,19 +91,103 @@ def forward_nvfp4(wl, x_bits, bias=None):
             "counts": counts.cpu().numpy(), "flags": flags}
 
 
-def oracle_outputs_nvfp4(wl, x_bits, tokens, r_oracle, batch=4):
+class HostExperts:
+    """Host copies of expert weights from the host generator, generated on a
+    thread pool (the generator's C calls release the GIL) and kept, least
+    recently used first out, within a byte budget of half the free memory."""
+
+    def __init__(self):
+        self.cache = collections.OrderedDict()  # (kind, H, I, E, e) -> (w13, w2)
+        self.bytes = 0
+
+    @staticmethod
+    def _make(kind, wl, e):
+        if kind == "bf16":
+            return synth.host_expert_w13(wl, e), synth.host_expert_w2(wl, e)
+        return synth.host_expert_w13_nvfp4(wl, e), synth.host_expert_w2_nvfp4(wl, e)
+
+    @staticmethod
+    def _nbytes(v):
+        return sum(a.nbytes for part in v for a in (part if isinstance(part, tuple) else (part,)))
+
+    def get(self, wl, experts, kind="bf16"):
+        """({e: w13}, {e: w2}) for the listed experts."""
+        want = sorted(set(int(e) for e in np.ravel(experts)))
+        keys = {e: (kind, wl.H, wl.I, wl.E, e) for e in want}
+        missing = [e for e in want if keys[e] not in self.cache]
+        if missing:
+            workers = max(1, min(16, os.cpu_count() or 1))
+            with concurrent.futures.ThreadPoolExecutor(workers) as pool:
+                made = list(pool.map(lambda e: self._make(kind, wl, e), missing))
+            for e, v in zip(missing, made):
+                self.cache[keys[e]] = v
+                self.bytes += self._nbytes(v)
+        for e in want:
+            self.cache.move_to_end(keys[e])
+        budget = psutil.virtual_memory().available // 2 + self.bytes
+        wanted = set(keys.values())
+        while self.bytes > budget:
+            k = next((k for k in self.cache if k not in wanted), None)
+            if k is None:
+                break
+            self.bytes -= self._nbytes(self.cache.pop(k))
+        w13 = {e: self.cache[keys[e]][0] for e in want}
+        w2 = {e: self.cache[keys[e]][1] for e in want}
+        return w13, w2
+
+
+HOST_EXPERTS = HostExperts()
+
+
+def _batches(tokens, ids, batch):
+    """Token batches in the order of their first expert, so that consecutive
+    batches share experts (fewer host weights generated per batch)."""
+    tokens = np.asarray(tokens)
+    order = tokens[np.argsort(ids[tokens, 0], kind="stable")]
+    for i in range(0, len(order), batch):
+        yield order[i:i + batch]
+
+
+def oracle_outputs_nvfp4(wl, x_bits, tokens, r_oracle, batch=64):
+    """Oracle output rows (NVFP4 expert path) for the listed tokens, in that order."""
     cfg = oracle.cfg_for(wl)
     g_w, g_a = synth.NVFP4_WEIGHT_SCALE, synth.NVFP4_ACT_SCALE
-    rows = []
-    for i in range(0, len(tokens), batch):
-        tt = np.asarray(tokens[i:i + batch])
+    out = {}
+    for tt in _batches(tokens, r_oracle["ids"], batch):
         ids = r_oracle["ids"][tt]
-        ex = sorted(set(int(v) for v in ids.ravel()))
-        w13 = {e: synth.host_expert_w13_nvfp4(wl, e) for e in ex}
-        w2 = {e: synth.host_expert_w2_nvfp4(wl, e) for e in ex}
-        rows.append(oracle.experts_nvfp4(cfg, x_bits[tt], ids, r_oracle["weights"][tt], w13, w2,
-                                         g_w, g_w, g_a, g_a))
-    return np.concatenate(rows, axis=0)
+        w13, w2 = HOST_EXPERTS.get(wl, ids, "nvfp4")
+        rows = oracle.experts_nvfp4(cfg, x_bits[tt], ids, r_oracle["weights"][tt], w13, w2,
+                                    g_w, g_w, g_a, g_a)
+        out.update(zip(tt.tolist(), rows))
+    return np.stack([out[int(t)] for t in tokens])
+
+
+def block_cover_tokens(ids, E, block, extra=0, seed=synth.SEED):
+    """Tokens whose rows cover, for every expert with rows, the first and last
+    rows of its first and last token blocks (rows of an expert are its tokens
+    in ascending order, cut into blocks of `block`), plus the first row of the
+    second half of its first block (where the second CTA of a pair starts);
+    then `extra` more tokens drawn at random. Sorted, without repeats."""
+    T, K = ids.shape
+    flat_e = ids.ravel()
+    flat_t = np.repeat(np.arange(T), K)
+    order = np.lexsort((flat_t, flat_e))
+    e_sorted, t_sorted = flat_e[order], flat_t[order]
+    starts = np.searchsorted(e_sorted, np.arange(E + 1))
+    pick = set()
+    for e in range(E):
+        c = starts[e + 1] - starts[e]
+        if c == 0:
+            continue
+        nb = (c + block - 1) // block
+        first_end = min(c, block)
+        for r in (0, first_end - 1, first_end // 2, (nb - 1) * block, c - 1):
+            pick.add(int(t_sorted[starts[e] + r]))
+    rng = np.random.default_rng(seed + 17)
+    rest = np.setdiff1d(np.arange(T), np.fromiter(pick, int, len(pick)))
+    if extra and rest.size:
+        pick.update(rng.choice(rest, size=min(extra, rest.size), replace=False).tolist())
+    return np.array(sorted(pick), dtype=np.int64)
 
 
 def to_dev_bits(a):
@@ -145,16 +234,25 @@ def check_routes(r_gpu, r_oracle, E):
     assert np.allclose(gw, ow, rtol=1e-5, atol=1e-6)
 
 
-def oracle_outputs(wl, x_bits, tokens, r_oracle, batch=4):
-    """Oracle output rows for the listed tokens, generating only their experts."""
+def oracle_outputs(wl, x_bits, tokens, r_oracle, batch=64):
+    """Oracle output rows for the listed tokens, in that order, generating only
+    their experts on the host."""
     cfg = oracle.cfg_for(wl)
-    rows = []
-    for i in range(0, len(tokens), batch):
-        tt = np.asarray(tokens[i:i + batch])
+    out = {}
+    for tt in _batches(tokens, r_oracle["ids"], batch):
         ids = r_oracle["ids"][tt]
-        w13, w2 = _inputs.expert_tables(wl, ids)
-        rows.append(oracle.experts(cfg, x_bits[tt], ids, r_oracle["weights"][tt], w13, w2))
-    return np.concatenate(rows, axis=0)
+        w13, w2 = HOST_EXPERTS.get(wl, ids)
+        rows = oracle.experts(cfg, x_bits[tt], ids, r_oracle["weights"][tt], w13, w2)
+        out.update(zip(tt.tolist(), rows))
+    return np.stack([out[int(t)] for t in tokens])
+
+
+def oracle_hidden(wl, x_bits, tokens, r_oracle):
+    """The oracle's silu(Wg x) * (Wu x) [len(tokens), K, I] for the listed tokens."""
+    cfg = oracle.cfg_for(wl)
+    ids = r_oracle["ids"][np.asarray(tokens)]
+    w13, _ = HOST_EXPERTS.get(wl, ids)
+    return oracle.hidden(cfg, x_bits[np.asarray(tokens)], ids, w13)
 
 
 def max_rel_err(out_bits, ref):

@@ -67,6 +67,7 @@ def test_workspace_size_scales_and_covers_intermediates():
     ("top_k", 129, INVALID),        # more experts than the kept groups hold
     ("renormalize", 2, INVALID),
     ("bias_mode", 3, INVALID),
+    ("router_tc", 2, INVALID),
     ("hidden", 5000, UNSUPPORTED),  # not a multiple of 128
     ("inter", 2500, UNSUPPORTED),
     ("n_experts", 1024, UNSUPPORTED),
@@ -194,3 +195,27 @@ def test_bench_describes_the_host_chunking_the_library_plans():
         fwd = up(max(ws_size(cfg, size, fwd_op)[1], ws_size(cfg, last, fwd_op)[1]))
         bufs = 1 if n == 1 else 2
         assert ws_size(cfg, T, host_op) == (OK, fwd + 2 * bufs * up(size * cfg.hidden * 2))
+
+
+def test_workspace_layout_rejects_bad_arguments_before_any_cuda_call():
+    cfg = bm.beam_cfg()
+    lay = bm.BeamMoeWsLayout()
+    L = bm.lib()
+    assert L.beam_moe_workspace_layout(ctypes.byref(cfg), 64, bm.OP_FORWARD_NVFP4,
+                                       ctypes.byref(lay)) == INVALID
+    assert L.beam_moe_workspace_layout(ctypes.byref(cfg), 64, bm.OP_FORWARD, None) == INVALID
+    assert L.beam_moe_workspace_layout(ctypes.byref(cfg), -1, bm.OP_FORWARD,
+                                       ctypes.byref(lay)) == INVALID
+
+
+def test_forward_stages_rejects_a_bad_stage_before_any_cuda_call():
+    cfg = bm.beam_cfg()
+    a = 1 << 20  # never dereferenced
+    ws_bytes = ws_size(cfg, 64)[1]
+    L = bm.lib()
+    for stage in (-1, 7):
+        assert L.beam_moe_forward_stages(ctypes.byref(cfg), 64, a, a, None, a, a, None, stage,
+                                         a, ws_bytes, None) == INVALID
+    # the whole forward needs an output
+    assert L.beam_moe_forward_stages(ctypes.byref(cfg), 64, a, a, None, a, a, None, 6, a,
+                                     ws_bytes, None) == INVALID

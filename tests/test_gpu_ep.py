@@ -93,7 +93,8 @@ def test_ep_tiny_many_rows(world, Ts):
 
 
 def test_ep_decode_full_size_eight_ranks():  # 32 experts per rank, 64 tokens each
-    _check(synth.workload("decode"), 8, [64] * 8, n_sample=12)
+    """Every output row of all eight ranks against the oracle."""
+    _check(synth.workload("decode"), 8, [64] * 8)
 
 
 @pytest.mark.parametrize("Ts", [[900, 600], [100, 37]])
@@ -106,3 +107,41 @@ def test_ep_return_address_out_of_range_is_dropped_and_flagged(Ts):
     GEMM ([100, 37]). Every access stays inside the workspaces, and the real
     rows' outputs still match the oracle."""
     _check(synth.workload("tiny"), 2, Ts, fill=0xFF, extra_rows=16, want_flags=0x400)
+
+
+def test_ep_dispatch_outside_the_receive_buffer_is_dropped_and_flagged():
+    """Rank 0 dispatches with a send_base that is not its plan: every row
+    shifted past the owners' receive capacity (as counts from another step
+    could place them), then every row at a negative place. No row is stored:
+    the peer's workspace is unchanged byte for byte, rank 0's own workspace
+    changes only in its status word and its combine positions, and status
+    bit 0x800 is set."""
+    wl = synth.workload("tiny")
+    world, Ts = 2, [100, 37]
+    cfg = _gpu.cfg_of(wl)
+    _, _, wr = _gpu.device_weights(wl)
+    x, _, _, b, _ = _inputs.routed_inputs(wl.with_T(sum(Ts)))
+    xs = np.split(x, np.cumsum(Ts)[:-1])
+    cap = sum(Ts) * wl.K
+    eps = [bm.ep_cfg(world, r, max(Ts), cap) for r in range(world)]
+    wss = [torch.empty(bm.beam_moe_ep_workspace_size(cfg, ep), dtype=torch.uint8, device="cuda")
+           for ep in eps]
+    for ws in wss:
+        ws.fill_(0x5A)
+        ws[:256].zero_()
+    peers = [ws.data_ptr() for ws in wss]
+    xd = [_gpu.to_dev_bits(v) for v in xs]
+    counts = [torch.empty(wl.E, dtype=torch.int32, device="cuda") for _ in range(world)]
+    for r in range(world):
+        bm.beam_moe_ep_route(cfg, eps[r], xd[r], wr, None, counts[r], wss[r])
+    counts_all = np.stack([c.cpu().numpy() for c in counts])
+    send_base = bm.beam_moe_ep_plan(cfg, eps[0], counts_all)[0]
+    for bad in (send_base + cap, np.full_like(send_base, -(1 << 20))):
+        before = [ws.cpu().numpy().copy() for ws in wss]
+        bm.beam_moe_ep_dispatch(cfg, eps[0], xd[0], torch.from_numpy(bad.astype(np.int32)).cuda(),
+                                peers, wss[0])
+        assert bm.beam_moe_check(wss[0]) == 0x800
+        after = [ws.cpu().numpy() for ws in wss]
+        assert np.array_equal(after[1], before[1])
+        changed = np.count_nonzero(after[0][256:] != before[0][256:])
+        assert changed <= Ts[0] * wl.K * 4  # the combine positions (-1 for every slot)

@@ -59,37 +59,35 @@ def test_nvfp4_forward_tiny(T):
     assert err <= _gpu.TOL, (err, rms)
 
 
-def test_nvfp4_decode_full_size():
-    wl = synth.workload("decode")
-    x, _, wr, b, r = _inputs.routed_inputs(wl)
-    g = _gpu.forward_nvfp4(wl, x)
-    assert g["flags"] == 0
-    _gpu.check_routes(g, r, wl.E)
-    tokens = synth.sample_tokens(wl.T, 12)
-    ref = _gpu.oracle_outputs_nvfp4(wl, x, tokens, r)
-    err, rms = _gpu.max_rel_err(g["out"][tokens], ref)
-    assert err <= _gpu.TOL, (err, rms)
-
-
-def _full_case(name, n_sample):
+def _full_case(name, tokens=None):
+    """Routing on every token; outputs on `tokens`, by default the tokens that
+    cover the first and last rows of every touched expert's first and last
+    128-row token tile (the NVFP4 GEMMs' tile; its 256-row pair tiles start on
+    every other one)."""
     wl = synth.workload(name)
     x, _, wr, b, r = _inputs.routed_inputs(wl)
     g = _gpu.forward_nvfp4(wl, x, bias=b)
     assert g["flags"] == 0
     _gpu.check_routes(g, r, wl.E)
-    tokens = synth.sample_tokens(wl.T, n_sample)
+    if tokens is None:
+        tokens = _gpu.block_cover_tokens(r["ids"], wl.E, 128)
     ref = _gpu.oracle_outputs_nvfp4(wl, x, tokens, r)
     err, rms = _gpu.max_rel_err(g["out"][tokens], ref)
     assert err <= _gpu.TOL, (err, rms)
 
 
+def test_nvfp4_decode_full_size():
+    """Every one of the 64 output rows."""
+    _full_case("decode", tokens=np.arange(64))
+
+
 def test_nvfp4_prefill_full_size():
-    _full_case("prefill", 8)
+    _full_case("prefill")
 
 
 def test_nvfp4_skewed_full_size():  # router bias on the logits of 16 hot experts
-    _full_case("skewed", 8)
+    _full_case("skewed")
 
 
 def test_nvfp4_long_full_size():  # 2048 rows per expert: the down GEMM runs on CTA pairs
-    _full_case("long", 8)
+    _full_case("long")

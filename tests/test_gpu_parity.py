@@ -5,7 +5,8 @@ same per-expert counts (inputs are re-drawn until every oracle top-k margin
 exceeds 1e-4, so fp32 and fp64 routing must agree). Outputs must match within
 max |err| <= 2e-2 x RMS of the oracle output (bf16 weights and activations,
 fp32 accumulation, bf16 h, fp32 y, bf16 out). Full-size workloads are compared on all
-routes and on sampled output rows.
+routes and on output rows that cover every touched expert's first and last token
+blocks (decode: every row).
 """
 import numpy as np
 import pytest
@@ -19,17 +20,24 @@ from tests import _gpu, _inputs
 pytestmark = pytest.mark.gpu
 
 
-def _full_case(name, n_sample):
+def _full_case(name, tokens=None, min_rows=0):
+    """Routing on every token; outputs on `tokens`, by default the tokens that
+    cover the first and last rows of every touched expert's first and last
+    256-row token block (the grouped GEMMs' token tiles, in both tile orders),
+    topped up at random to at least `min_rows` rows."""
     wl = synth.workload(name)
     x, _, wr, b, r = _inputs.routed_inputs(wl)
     g = _gpu.forward(wl, x, bias=b)
     assert g["flags"] == 0
     _gpu.check_routes(g, r, wl.E)
-    tokens = synth.sample_tokens(wl.T, n_sample)
+    if tokens is None:
+        tokens = _gpu.block_cover_tokens(r["ids"], wl.E, 256)
+        if len(tokens) < min_rows:
+            tokens = _gpu.block_cover_tokens(r["ids"], wl.E, 256, extra=min_rows - len(tokens))
     ref = _gpu.oracle_outputs(wl, x, tokens, r)
     err, rms = _gpu.max_rel_err(g["out"][tokens], ref)
     assert err <= _gpu.TOL, (name, err, rms)
-    return wl, x, r, g
+    return wl, x, r, g, tokens
 
 
 def test_device_generator_matches_host():
@@ -181,18 +189,23 @@ def test_route_only_entry_point():
 
 
 def test_decode_full_size():
-    _full_case("decode", 16)
+    """Every one of the 64 output rows."""
+    _full_case("decode", tokens=np.arange(64))
 
 
 def test_prefill_full_size():
-    _full_case("prefill", 24)
+    *_, tokens = _full_case("prefill", min_rows=512)
+    assert len(tokens) >= 512
 
 
 def test_skewed_full_size():
-    wl, x, r, g = _full_case("skewed", 24)
+    wl, x, r, g, tokens = _full_case("skewed")
     hot = synth.hot_experts(wl)
     assert g["counts"][hot].sum() > 0.5 * wl.T * wl.K  # the 16 hot experts take most rows
+    # experts with more rows than weight rows run token block by token block,
+    # the others weight block by weight block: both orders are compared
+    assert g["counts"].max() > 2 * wl.I and np.any((g["counts"] > 0) & (g["counts"] <= 2 * wl.I))
 
 
 def test_long_full_size():
-    _full_case("long", 24)
+    _full_case("long")
