@@ -506,6 +506,134 @@ def measure(args, wl, ex, dev, stream, rank, world, local):
     return part
 
 
+def run_ep(args, wl):
+    """Expert parallelism over the N ranks (one per GPU; N = 1 runs the same
+    phases on one GPU): each rank holds E / N experts, routes its own T
+    tokens, exchanges workspaces once through CUDA IPC, and per step
+    all-gathers the counts (NCCL), plans on the host, dispatches by peer
+    stores, runs its experts (y rows stored back into their sources) and
+    combines, with a barrier after the dispatch and after the experts."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import sparse_moe_layer_beam_b200 as bm
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if wl.E % world:
+        raise SystemExit(f"{wl.E} experts do not split over {world} ranks")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    stream = torch.cuda.current_stream()
+    st = stream.cuda_stream
+    ex = Experts(wl, "bf16", dev, st)
+    cfg = bm.beam_cfg(wl.H, wl.I, wl.E, wl.G, wl.Gk, wl.K, wl.renormalize, args.bias_mode,
+                      wl.scale, router_tc=args.router_tc)
+    El = wl.E // world
+    w13 = ex.w13.data_ptr() + rank * El * 2 * wl.I * wl.H * 2
+    w2 = ex.w2.data_ptr() + rank * El * wl.H * wl.I * 2
+    bias = synth.host_bias(wl)
+    b = None if bias is None else torch.from_numpy(bias).to(dev)
+    x = torch.empty((wl.T, wl.H), dtype=torch.int16, device=dev)
+    synth.dev_x(wl, x.data_ptr(), st, seed=rank_seed(rank))
+    out = torch.empty((wl.T, wl.H), dtype=torch.int16, device=dev)
+    ep = bm.ep_cfg(world, rank, wl.T, wl.T * world * min(wl.K, El))
+    ws = torch.empty(bm.beam_moe_ep_workspace_size(cfg, ep), dtype=torch.uint8, device=dev)
+    counts = torch.empty(wl.E, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    if world > 1:
+        peers = bm.EpPeers(ep, ws, bm.torch_gather())
+        gathered = [torch.empty_like(counts) for _ in range(world)]
+        ones = torch.ones(1, device=dev)
+    else:
+        peers = bm.EpPeers(ep, ws, lambda blob: [blob], export=lambda w: b"self")
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.all_reduce(ones)  # stream-ordered: every rank's earlier work is done
+
+    def step():
+        bm.beam_moe_ep_route(cfg, ep, x, ex.wr, b, counts, ws, stream=st)
+        if world > 1:
+            dist.all_gather(gathered, counts)
+            counts_all = torch.stack(gathered).cpu().numpy()
+        else:
+            counts_all = counts.cpu().numpy()[None]
+        send_base, recv_counts, _ = bm.beam_moe_ep_plan(cfg, ep, counts_all)
+        bm.beam_moe_ep_dispatch(cfg, ep, x, torch.from_numpy(send_base).to(dev, non_blocking=True),
+                                peers.ptrs, ws, stream=st)
+        barrier()
+        bm.beam_moe_ep_experts(cfg, ep, recv_counts, w13, w2, peers.ptrs, ws, stream=st)
+        barrier()
+        bm.beam_moe_ep_combine(cfg, ep, wl.T, out, ws, stream=st)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    if bm.beam_moe_check(ws, st):
+        raise SystemExit("device status flags after warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    flags = bm.beam_moe_check(ws, st)
+    if flags:
+        raise SystemExit(f"device status flags {flags:#x} in the timed region")
+    total_ms = max_over_ranks([sum(a.elapsed_time(c) for a, c in ev)], dev)[0]
+    ms_step = total_ms / args.steps
+    value = wl.T * world / (ms_step / 1000.0)
+    alg = algorithmic(wl, counts.cpu().numpy(), "bf16")
+    peaks, peak_kind = load_peaks()
+    _, block = roofline(alg, None, ms_step, peaks, peak_kind, False)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(wl) + " [expert parallel]", "T": wl.T,
+                   "tokens_per_rank": wl.T, "experts_per_rank": El,
+                   "l2": "flushed before every timed step (256 MB write, outside the events)",
+                   "parallelism": f"expert parallel x{world}: peer-store dispatch and return "
+                                  "through CUDA IPC, NCCL all-gather of counts"},
+        "roofline": None, "block": block, "clocks": clk,
+        # router GEMM, top-k, scan, dispatch, gate/up, down (+ the return copy
+        # when the down GEMM runs on single CTAs, below 64 rows per expert),
+        # combine; the tensor-core router adds its weight split
+        "gpu_launches": (7 + (1 if wl.T * world * wl.K / wl.E < 64 else 0)
+                         + (1 if args.router_tc else 0)) * args.steps,
+    }
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    peers.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # The default run times every Beam workload; the line's headline is the last
 # (the long prefill chunk, the largest configuration that fits one GPU).
 DEFAULT_WORKLOADS = ("decode", "prefill", "skewed", "long")
@@ -574,6 +702,8 @@ def main():
                     help="opt in to the router GEMM on tensor cores (exact bf16 split)")
     ap.add_argument("--replay", action="store_true",
                     help="time the expert path with recorded routes (beam_moe_forward_routed)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism over the N ranks (one workload, bf16)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (small profiling captures only)")
     ap.add_argument("--experts", type=int, default=None,
@@ -595,6 +725,10 @@ def main():
         wls.append(wl)
     if args.impl == "reference":
         return run_reference(args, wls[-1])
+    if args.ep:
+        if len(wls) != 1 or args.format != "bf16" or args.replay:
+            raise SystemExit("--ep times one bf16 workload (--workload decode, ...)")
+        return run_ep(args, wls[0])
     return run_ours(args, wls)
 
 

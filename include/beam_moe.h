@@ -402,6 +402,44 @@ BEAM_MOE_API beam_moe_status beam_moe_ep_combine(const beam_moe_cfg* cfg,
                                                  void* stream);
 
 /*
+ * Peer workspaces across processes (one process per GPU), through CUDA IPC.
+ * Each rank exports its workspace once, the ranks exchange the handles (any
+ * all-gather of these bytes; sizeof(beam_moe_ep_handle) is fixed), and each
+ * rank imports every other rank's handle to get the peer_ws pointers the
+ * dispatch and experts calls store through.
+ *   beam_moe_ep_export  ws: this rank's workspace, device memory from
+ *                       cudaMalloc (torch's default allocator qualifies; the
+ *                       virtual-memory allocator's expandable segments do
+ *                       not), at least ws_bytes long. Fills *handle: the IPC
+ *                       handle of the allocation holding ws, ws's offset in
+ *                       it, ws_bytes, the device ordinal and the process id.
+ *   beam_moe_ep_import  opens another process's handle on the current device
+ *                       (peer access is enabled as needed) and returns its
+ *                       workspace in *peer_ws. A handle this process exported
+ *                       is refused (BEAM_MOE_ERR_INVALID_ARG): use the local
+ *                       pointer for your own rank. ws_bytes must not exceed
+ *                       the exported size.
+ *   beam_moe_ep_release closes what beam_moe_ep_import opened (peer_ws as it
+ *                       returned it, with the same handle). Release every
+ *                       peer before the exporting process frees or exits.
+ * These calls synchronize with the device as CUDA IPC does; make them once at
+ * set-up, not per step.
+ */
+typedef struct beam_moe_ep_handle {
+  uint8_t ipc[64];  /* cudaIpcMemHandle_t of the allocation holding ws        */
+  int64_t offset;   /* ws minus the allocation's base, bytes                  */
+  int64_t bytes;    /* exported workspace size                                */
+  int32_t device;   /* exporting device ordinal                               */
+  int32_t pid;      /* exporting process                                      */
+} beam_moe_ep_handle;
+BEAM_MOE_API beam_moe_status beam_moe_ep_export(void* ws, size_t ws_bytes,
+                                                beam_moe_ep_handle* handle);
+BEAM_MOE_API beam_moe_status beam_moe_ep_import(const beam_moe_ep_handle* handle,
+                                                size_t ws_bytes, void** peer_ws);
+BEAM_MOE_API beam_moe_status beam_moe_ep_release(const beam_moe_ep_handle* handle,
+                                                 void* peer_ws);
+
+/*
  * Synchronizes `stream`, then reads and clears the device status word in the
  * workspace. *device_flags (may be NULL) receives the raw bits: 0x1 producer,
  * 0x2 MMA issuer, 0x4 epilogue gave up a bounded wait; 0x100 an expert id

@@ -24,6 +24,8 @@ __all__ = ["BeamMoeCfg", "BeamMoeError", "Trace", "OP_ROUTE", "OP_FORWARD", "N_S
            "beam_moe_ep_combine", "beam_moe_selftest_wait",
            "beam_moe_forward", "beam_moe_forward_routed", "beam_moe_forward_traced",
            "beam_moe_forward_stages", "beam_moe_workspace_layout", "BeamMoeWsLayout",
+           "BeamMoeEpHandle", "beam_moe_ep_export", "beam_moe_ep_import",
+           "beam_moe_ep_release", "EpPeers", "torch_gather",
            "beam_moe_check"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -71,6 +73,12 @@ class BeamMoeEpCfg(ctypes.Structure):
                 ("recv_cap", ctypes.c_int64)]
 
 
+class BeamMoeEpHandle(ctypes.Structure):
+    """A workspace exported for other processes (CUDA IPC handle and offset)."""
+    _fields_ = [("ipc", ctypes.c_uint8 * 64), ("offset", ctypes.c_int64),
+                ("bytes", ctypes.c_int64), ("device", ctypes.c_int32), ("pid", ctypes.c_int32)]
+
+
 class BeamMoeError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
@@ -114,6 +122,10 @@ _SIGS = {
     "beam_moe_ep_dispatch": [_CFG, _EP, ctypes.c_int64, _P, _P, _PP, _P, ctypes.c_size_t, _P],
     "beam_moe_ep_experts": [_CFG, _EP, _P, _P, _P, _PP, _P, ctypes.c_size_t, _P],
     "beam_moe_ep_combine": [_CFG, _EP, ctypes.c_int64, _P, _P, ctypes.c_size_t, _P],
+    "beam_moe_ep_export": [_P, ctypes.c_size_t, ctypes.POINTER(BeamMoeEpHandle)],
+    "beam_moe_ep_import": [ctypes.POINTER(BeamMoeEpHandle), ctypes.c_size_t,
+                           ctypes.POINTER(ctypes.c_void_p)],
+    "beam_moe_ep_release": [ctypes.POINTER(BeamMoeEpHandle), _P],
     "beam_moe_trace_create": [ctypes.c_int32, ctypes.POINTER(_P)],
     "beam_moe_trace_destroy": [_P],
     "beam_moe_trace_reset": [_P],
@@ -394,3 +406,72 @@ def beam_moe_ep_combine(cfg, ep, T, out, ws, stream=None):
     _check(lib().beam_moe_ep_combine(ctypes.byref(cfg), ctypes.byref(ep), T, _ptr(out), _ptr(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)),
            "beam_moe_ep_combine")
+
+
+def beam_moe_ep_export(ws):
+    """This rank's workspace as bytes another process can import."""
+    h = BeamMoeEpHandle()
+    _check(lib().beam_moe_ep_export(_ptr(ws), ws.numel() * ws.element_size(), ctypes.byref(h)),
+           "beam_moe_ep_export")
+    return bytes(h)
+
+
+def beam_moe_ep_import(blob, ws_bytes):
+    """Device address of another process's exported workspace."""
+    h = BeamMoeEpHandle.from_buffer_copy(blob)
+    p = ctypes.c_void_p(0)
+    _check(lib().beam_moe_ep_import(ctypes.byref(h), ws_bytes, ctypes.byref(p)),
+           "beam_moe_ep_import")
+    return p.value
+
+
+def beam_moe_ep_release(blob, peer_ws):
+    h = BeamMoeEpHandle.from_buffer_copy(blob)
+    _check(lib().beam_moe_ep_release(ctypes.byref(h), peer_ws), "beam_moe_ep_release")
+
+
+class EpPeers:
+    """Every rank's workspace as an address this process can store to.
+
+    gather(blob) must return the list of every rank's blob in rank order (an
+    all-gather, e.g. torch.distributed.all_gather_object); export / import_ /
+    release default to the library's CUDA IPC calls. This rank's own slot is
+    its local workspace; every other slot is imported, and close() releases
+    them (call it on every rank, after a barrier, before any rank frees its
+    workspace)."""
+
+    def __init__(self, ep, ws, gather, export=None, import_=None, release=None):
+        self._release = release or beam_moe_ep_release
+        mine = (export or beam_moe_ep_export)(ws)
+        blobs = gather(mine)
+        if len(blobs) != ep.world or blobs[ep.rank] != mine:
+            raise ValueError("gather must return every rank's blob in rank order")
+        nbytes = ws.numel() * ws.element_size()
+        self.ptrs, self._opened = [], []
+        try:
+            for r, blob in enumerate(blobs):
+                if r == ep.rank:
+                    self.ptrs.append(ws.data_ptr())
+                else:
+                    p = (import_ or beam_moe_ep_import)(blob, nbytes)
+                    self._opened.append((blob, p))
+                    self.ptrs.append(p)
+        except Exception:
+            self.close()
+            raise
+
+    def close(self):
+        while self._opened:
+            blob, p = self._opened.pop()
+            self._release(blob, p)
+
+
+def torch_gather(group=None):
+    """An all-gather of Python objects over a torch.distributed group."""
+    import torch.distributed as dist
+
+    def gather(obj):
+        out = [None] * dist.get_world_size(group)
+        dist.all_gather_object(out, obj, group=group)
+        return out
+    return gather

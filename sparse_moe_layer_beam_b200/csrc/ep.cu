@@ -111,6 +111,8 @@ __global__ void __launch_bounds__(128) ep_dispatch_kernel(
     if (!d) continue;
     for (int v = tid; v < H / 8; v += 128) d[v] = __ldg(src + v);
   }
+  // the owners read these rows in their next phase, on other GPUs
+  __threadfence_system();
 }
 
 // Every received y row back to its source rank's returned-y buffer.
@@ -132,6 +134,7 @@ __global__ void __launch_bounds__(128) ep_return_kernel(const float* __restrict_
     const float4* from = reinterpret_cast<const float4*>(y + (size_t)i * H);
     for (int v = threadIdx.x; v < H / 4; v += 128) d[v] = __ldg(from + v);
   }
+  __threadfence_system();  // the sources combine these rows on other GPUs
 }
 
 }  // namespace

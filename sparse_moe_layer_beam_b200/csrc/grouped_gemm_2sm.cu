@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (EPRET) __threadfence_system();  // the sources combine these rows on other GPUs
   }
   __syncwarp();
   tc_fence_before();

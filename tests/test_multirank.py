@@ -115,3 +115,81 @@ def test_expert_parallel_plan_over_gloo():
     assert ok0 and ok1
     assert tot0 == tot1 == (50 + 80) * 8        # every assignment of both ranks
     assert rows0 + rows1 == tot0                 # received exactly once, by its owner
+
+
+class _FakeWs:
+    """Stands in for a workspace tensor on a CPU-only rank."""
+
+    def __init__(self, addr, nbytes):
+        self.addr, self.nbytes = addr, nbytes
+
+    def data_ptr(self):
+        return self.addr
+
+    def numel(self):
+        return self.nbytes
+
+    def element_size(self):
+        return 1
+
+
+def _ipc_worker(rank, world, port, out):
+    """The peer-workspace exchange over a real process group (gloo): every rank
+    exports, the blobs are all-gathered, every other rank's blob is imported
+    once, the own slot stays local, and close() releases exactly what was
+    opened. Export / import / release are fakes (no GPU here); the library's
+    CUDA IPC calls are exercised by the GPU test with two processes."""
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import sparse_moe_layer_beam_b200 as bm
+
+    imported, released = [], []
+
+    def export(ws):
+        return f"ws-of-{rank}-at-{ws.data_ptr()}".encode()
+
+    def import_(blob, nbytes):
+        imported.append((blob, nbytes))
+        return 10_000 + int(blob.decode().split("-")[2])
+
+    def release(blob, p):
+        released.append((blob, p))
+
+    ep = bm.ep_cfg(world, rank, 64, 1024)
+    ws = _FakeWs(4096 * (rank + 1), 777)
+    peers = bm.EpPeers(ep, ws, bm.torch_gather(), export, import_, release)
+    ptrs = list(peers.ptrs)
+    peers.close()
+    bad = None
+    try:  # a gather that returns the blobs out of rank order is refused
+        rotate = lambda b: (lambda v: v[1:] + v[:1])(bm.torch_gather()(b))  # noqa: E731
+        bm.EpPeers(ep, ws, rotate, export, import_, release)
+    except ValueError as e:
+        bad = str(e)
+    out.put((rank, ptrs, [b.decode() for b, _ in imported], [p for _, p in released], bad))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_expert_parallel_peer_exchange_over_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 32500 + os.getpid() % 1000
+    world = 3
+    procs = [ctx.Process(target=_ipc_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ptrs, imported, released, bad in res:
+        assert ptrs[rank] == 4096 * (rank + 1)  # the own slot is the local workspace
+        others = [r for r in range(world) if r != rank]
+        assert [ptrs[r] for r in others] == [10_000 + r for r in others]
+        assert imported[:world - 1] == [f"ws-of-{r}-at-{4096 * (r + 1)}" for r in others]
+        assert sorted(released) == sorted(10_000 + r for r in others)
+        assert bad and "rank order" in bad
