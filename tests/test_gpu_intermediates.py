@@ -138,7 +138,8 @@ def _check_h(wl, x, r, ids, pos, ws, lay, tokens):
     assert misrounded <= MAX_MISROUNDED
 
 
-@pytest.mark.parametrize("T", [300, 1500])  # 1-CTA tiles; CTA pairs (>= 64 rows per expert)
+# 1-CTA tiles; CTA pairs (>= 64 rows per expert); 512-token pair tiles (>= 512)
+@pytest.mark.parametrize("T", [300, 1500, 2100])
 def test_tiny_intermediates(T):
     wl = synth.workload("tiny").with_T(T)
     x, _, wr, b, r = _inputs.routed_inputs(wl)
@@ -146,7 +147,8 @@ def test_tiny_intermediates(T):
     ids, pos = _check_dispatch(wl, x, r, ws, lay)
     _check_permuted_rows(wl, x, pos, ws, lay)
     ws, lay = _run_stages(wl, x, 4)
-    assert lay.pair_gateup == (1 if T == 1500 else 0)
+    assert lay.pair_gateup == (1 if T >= 1500 else 0)
+    assert lay.pair_wide == (1 if T >= 2100 else 0)
     _check_h(wl, x, r, ids, pos, ws, lay, np.arange(T))
 
 

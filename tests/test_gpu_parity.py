@@ -85,11 +85,13 @@ def test_tiny_ragged_token_counts(T):
     assert err <= _gpu.TOL, err
 
 
-@pytest.mark.parametrize("T", [600, 1024, 1500])
+@pytest.mark.parametrize("T", [600, 1024, 1500, 2100, 3001])
 def test_tiny_many_rows_per_expert(T):
     """More than 100 rows per expert on average: the grouped GEMMs run on CTA
     pairs (cta_group::2) with ragged token blocks, each CTA loading its half
-    of a block's rows as a box of 64 or 128 rows."""
+    of a block's rows as a box of 64 or 128 rows. From 512 rows per expert
+    (T = 2100, 3001) the tiles are 512 tokens wide, two accumulators per
+    weight tile, the second one empty in tiles with at most 256 rows."""
     wl = synth.workload("tiny").with_T(T)
     x, _, wr, b, r = _inputs.routed_inputs(wl)
     g = _gpu.forward(wl, x)
