@@ -634,6 +634,68 @@ def run_ep(args, wl):
     return 0
 
 
+def run_route_only(args, wl):
+    """Routing alone (beam_moe_route: router GEMM, top-k and the per-expert
+    counts) on one GPU, with no expert weights allocated: the router's own
+    throughput, against the FP32 ALU peak (2 H E FLOP per token of FMAs)."""
+    import torch
+
+    import sparse_moe_layer_beam_b200 as bm
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    st = stream.cuda_stream
+    cfg = bm.beam_cfg(wl.H, wl.I, wl.E, wl.G, wl.Gk, wl.K, wl.renormalize, args.bias_mode,
+                      wl.scale, router_tc=args.router_tc)
+    wr = torch.from_numpy(synth.host_router(wl)).to(dev)
+    bias = synth.host_bias(wl)
+    b = None if bias is None else torch.from_numpy(bias).to(dev)
+    x = torch.empty((wl.T, wl.H), dtype=torch.int16, device=dev)
+    synth.dev_x(wl, x.data_ptr(), st)
+    ids = torch.empty((wl.T, wl.K), dtype=torch.int32, device=dev)
+    w = torch.empty((wl.T, wl.K), dtype=torch.float32, device=dev)
+    counts = torch.empty(wl.E, dtype=torch.int32, device=dev)
+    ws = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T, bm.OP_ROUTE), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        bm.beam_moe_route(cfg, x, wr, b, ids, w, counts, ws, stream=st)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(0)
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        bm.beam_moe_route(cfg, x, wr, b, ids, w, counts, ws, stream=st)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if bm.beam_moe_check(ws, st):
+        raise SystemExit("device status flags in the timed region")
+    ms = sum(a.elapsed_time(c) for a, c in ev) / args.steps
+    flops = 2.0 * wl.H * wl.E * wl.T
+    lay = bm.beam_moe_workspace_layout(cfg, wl.T, bm.OP_ROUTE)
+    line = {
+        "metric": "router tokens/s (beam_moe_route)", "value": wl.T / (ms / 1000.0),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": describe(wl) + " [routing only]", "T": wl.T,
+                   "router": "tensor cores (exact bf16 split)" if lay.router_tc
+                   else "FP32 FMA on CUDA cores", "router_splits": lay.router_splits,
+                   "l2": "flushed before every timed step (256 MB write, outside the events)"},
+        "router_tflops": flops / (ms / 1000.0) / 1e12,
+        "gpu_launches": (4 if lay.router_tc else 3) * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # The default run times every Beam workload; the line's headline is the last
 # (the long prefill chunk, the largest configuration that fits one GPU).
 DEFAULT_WORKLOADS = ("decode", "prefill", "skewed", "long")
@@ -704,6 +766,8 @@ def main():
                     help="time the expert path with recorded routes (beam_moe_forward_routed)")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism over the N ranks (one workload, bf16)")
+    ap.add_argument("--route-only", action="store_true",
+                    help="time beam_moe_route alone on one workload (no expert weights)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (small profiling captures only)")
     ap.add_argument("--experts", type=int, default=None,
@@ -725,6 +789,10 @@ def main():
         wls.append(wl)
     if args.impl == "reference":
         return run_reference(args, wls[-1])
+    if args.route_only:
+        if len(wls) != 1 or args.gpus != 1:
+            raise SystemExit("--route-only times one workload on one GPU")
+        return run_route_only(args, wls[0])
     if args.ep:
         if len(wls) != 1 or args.format != "bf16" or args.replay:
             raise SystemExit("--ep times one bf16 workload (--workload decode, ...)")

@@ -46,23 +46,16 @@ __device__ __forceinline__ void decode_tile(int tile, const GemmParams& p, int& 
   nb = local - mb * nblk;
 }
 
-// silu(g) u in FP32 for the bf16 path: silu(g) = g / (1 + e^-g) with the
-// hardware exponential and an approximate FP32 division, both within a few
-// FP32 ulps, so h = silu(g) u is FP32-accurate before its one bf16 rounding
-// (the SwiGLU product is FP32 in "Welcome Beam", section "Residual Stream").
-// For g below about -88, e^-g overflows to +inf and the quotient is -0.
+// silu(g) u in FP32: silu(g) = g / (1 + e^-g) with the hardware exponential
+// and an approximate FP32 division, both within a few FP32 ulps, so h =
+// silu(g) u is FP32-accurate before it is rounded to bf16 or quantised to
+// NVFP4 (the SwiGLU product is FP32 in "Welcome Beam", section "Residual
+// Stream"). A cheaper tanh form (relative error 2^-11) moved h across
+// rounding and E2M1 quantisation boundaries often enough to show in the
+// output. For g below about -88, e^-g overflows to +inf and the quotient is
+// -0.
 __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fdividef(g, 1.0f + __expf(-g)) * u;
-}
-
-// silu(g) u for the NVFP4 path, where h is quantised to E2M1 (4 bits) next:
-// silu(g) = (g/2)(1 + tanh(g/2)) with one hardware tanh (relative error about
-// 2^-11), far below the E2M1 step, instead of an exponential and a division.
-__device__ __forceinline__ float silu_mul_fast(float g, float u) {
-  const float hg = 0.5f * g;
-  float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hg));
-  return fmaf(hg, t, hg) * u;
 }
 
 }  // namespace gg

@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(Cfg4<GATEUP>::kThreads, 1)
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              hb[j] = __float_as_uint(gg::silu_mul_fast(__uint_as_float(g[j]) * p.acc_scale,
+              hb[j] = __float_as_uint(gg::silu_mul(__uint_as_float(g[j]) * p.acc_scale,
                                                    __uint_as_float(u[j]) * p.acc_scale));
             tmem_st16(tp + 16 * c, hb);
           }
