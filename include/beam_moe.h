@@ -290,7 +290,6 @@ typedef struct beam_moe_ws_layout {
   int32_t router_tc;     /* 1: the router GEMM runs on tensor cores           */
   int32_t pair_gateup;   /* 1: gate/up grouped GEMM on CTA pairs              */
   int32_t pair_down;     /* 1: down grouped GEMM on CTA pairs                 */
-  int32_t pair_wide;     /* 1: both grouped GEMMs on CTA pairs, 512-token tiles */
 } beam_moe_ws_layout;
 BEAM_MOE_API beam_moe_status beam_moe_workspace_layout(const beam_moe_cfg* cfg, int64_t T,
                                                        beam_moe_op op,

@@ -68,10 +68,7 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool allow_tc) {
   const bool pair_ok = L.bn == 256 && pair_gemm_supported(c);
   L.pair_gateup = (pair_ok && mean_rows >= 64.0) ? 1 : 0;
   L.pair_down = (pair_ok && mean_rows >= 64.0) ? 1 : 0;
-  // From 512 rows per expert on average, tiles of 512 tokens (two
-  // accumulators per weight tile) cut the operand bytes each SM reads per
-  // FLOP by a quarter; below that most tiles would fill one accumulator.
-  L.pair_wide = (pair_ok && mean_rows >= 512.0) ? 1 : 0;
+
   size_t o = 0;
   auto take = [&](size_t bytes, size_t align) {
     o = align_up(o, align);
@@ -292,14 +289,12 @@ beam_moe_status expert_path(const beam_moe_cfg* cfg, const Layout& L, const uint
   BEAM_CUDA(beam::launch_permute(*cfg, L, x, ws, st));
   BEAM_CUDA(rec.mark(4));
   if (last < 4) return BEAM_MOE_OK;
-  BEAM_CUDA(L.pair_wide     ? beam::launch_gateup_wide(*cfg, L, w13, ws, st)
-            : L.pair_gateup ? beam::launch_gateup_pair(*cfg, L, w13, ws, st)
-                            : beam::launch_gateup(*cfg, L, w13, ws, st));
+  BEAM_CUDA(L.pair_gateup ? beam::launch_gateup_pair(*cfg, L, w13, ws, st)
+                          : beam::launch_gateup(*cfg, L, w13, ws, st));
   BEAM_CUDA(rec.mark(5));
   if (last < 5) return BEAM_MOE_OK;
-  BEAM_CUDA(L.pair_wide   ? beam::launch_down_wide(*cfg, L, w2, ws, st)
-            : L.pair_down ? beam::launch_down_pair(*cfg, L, w2, ws, st)
-                          : beam::launch_down(*cfg, L, w2, ws, st));
+  BEAM_CUDA(L.pair_down ? beam::launch_down_pair(*cfg, L, w2, ws, st)
+                        : beam::launch_down(*cfg, L, w2, ws, st));
   BEAM_CUDA(rec.mark(6));
   if (last < 6) return BEAM_MOE_OK;
   BEAM_CUDA(beam::launch_combine(*cfg, L, out, ws, st));
@@ -661,7 +656,6 @@ beam_moe_status beam_moe_workspace_layout(const beam_moe_cfg* cfg, int64_t T, be
   out->router_tc = L.router_tc;
   out->pair_gateup = L.pair_gateup;
   out->pair_down = L.pair_down;
-  out->pair_wide = L.pair_wide;
   return BEAM_MOE_OK;
 }
 

@@ -78,7 +78,6 @@ struct Layout {
   int bn;           // token tile of the grouped GEMMs
   int pair_gateup; // 1: gate/up grouped GEMM on CTA pairs
   int pair_down;   // 1: down grouped GEMM on CTA pairs
-  int pair_wide;   // 1: both grouped GEMMs on CTA pairs with 512-token tiles
   size_t status;    // uint32[64]
   size_t counts;    // int32[E]
   size_t offsets;   // int32[E + 1] first row of each expert in the permuted rows
@@ -179,12 +178,6 @@ cudaError_t launch_gateup_pair(const beam_moe_cfg& c, const Layout& L, const uin
                                char* ws, cudaStream_t st);
 cudaError_t launch_down_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2,
                              char* ws, cudaStream_t st, const EpReturn* ret = nullptr);
-// 512-token pair tiles (two accumulators sharing each weight tile); need
-// L.bn == 256, so that L.nb2_off counts 512-row blocks.
-cudaError_t launch_gateup_wide(const beam_moe_cfg& c, const Layout& L, const uint16_t* w13,
-                               char* ws, cudaStream_t st);
-cudaError_t launch_down_wide(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2, char* ws,
-                             cudaStream_t st);
 cudaError_t launch_combine(const beam_moe_cfg& c, const Layout& L, uint16_t* out, char* ws,
                            cudaStream_t st);
 cudaError_t launch_copy_routes(const beam_moe_cfg& c, const Layout& L, int32_t* ids_out,

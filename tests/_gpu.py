@@ -255,6 +255,25 @@ def oracle_hidden(wl, x_bits, tokens, r_oracle):
     return oracle.hidden(cfg, x_bits[np.asarray(tokens)], ids, w13)
 
 
+# NVFP4 outputs, beyond their own bf16 rounding: max |err| - half a bf16 step
+# of the output <= TOL_NVFP4 x RMS. The block's tolerance of 2e-2 x RMS is
+# stated for BF16 weights and activations; NVFP4 outputs have heavier tails
+# (RMS about 1.75, elements up to about 20 at Beam's shapes), where half a
+# bf16 step alone (1/32 in [8, 16), 1/16 in [16, 32)) exceeds 2e-2 x RMS. The
+# rest of the NVFP4 arithmetic (x and h quantised by the same rule on both
+# sides, FP32 against fp64 sums) is held to 1e-2 x RMS.
+TOL_NVFP4 = 1e-2
+
+
+def nvfp4_excess(out_bits, ref):
+    """(max over elements of (|err| - half a bf16 step at the output) / RMS, RMS)."""
+    got = synth.bf16_to_f32(out_bits).astype(np.float64)
+    rms = np.sqrt(np.mean(ref ** 2))
+    _, e = np.frexp(np.maximum(np.abs(ref), np.abs(got)))
+    half_step = np.ldexp(1.0, e - 9)  # bf16 keeps 8 significant bits
+    return ((np.abs(got - ref) - half_step) / rms).max(), rms
+
+
 def max_rel_err(out_bits, ref):
     got = synth.bf16_to_f32(out_bits).astype(np.float64)
     rms = np.sqrt(np.mean(ref ** 2))

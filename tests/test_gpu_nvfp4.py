@@ -1,7 +1,8 @@
 """NVFP4 (W4A4) path against the oracle: the GPU quantiser bit for bit (scales
 exactly, values exactly), the device weight fill against the host generator,
-and the whole block (routing bit-exact, outputs within 2e-2 x RMS of the
-oracle's fp64 evaluation on exactly dequantised values)."""
+and the whole block (routing bit-exact; outputs against the oracle's fp64
+evaluation on exactly dequantised values within half a bf16 step of the
+output plus 1e-2 x RMS, see _gpu.TOL_NVFP4)."""
 import numpy as np
 import pytest
 import torch
@@ -55,8 +56,8 @@ def test_nvfp4_forward_tiny(T):
     _gpu.check_routes(g, r, wl.E)
     tokens = np.arange(wl.T) if wl.T <= 256 else synth.sample_tokens(wl.T, 64)
     ref = _gpu.oracle_outputs_nvfp4(wl, x, tokens, r, batch=64)
-    err, rms = _gpu.max_rel_err(g["out"][tokens], ref)
-    assert err <= _gpu.TOL, (err, rms)
+    err, rms = _gpu.nvfp4_excess(g["out"][tokens], ref)
+    assert err <= _gpu.TOL_NVFP4, (err, rms)
 
 
 def _full_case(name, tokens=None):
@@ -72,8 +73,8 @@ def _full_case(name, tokens=None):
     if tokens is None:
         tokens = _gpu.block_cover_tokens(r["ids"], wl.E, 128)
     ref = _gpu.oracle_outputs_nvfp4(wl, x, tokens, r)
-    err, rms = _gpu.max_rel_err(g["out"][tokens], ref)
-    assert err <= _gpu.TOL, (err, rms)
+    err, rms = _gpu.nvfp4_excess(g["out"][tokens], ref)
+    assert err <= _gpu.TOL_NVFP4, (err, rms)
 
 
 def test_nvfp4_decode_full_size():

@@ -89,9 +89,9 @@ def test_tiny_ragged_token_counts(T):
 def test_tiny_many_rows_per_expert(T):
     """More than 100 rows per expert on average: the grouped GEMMs run on CTA
     pairs (cta_group::2) with ragged token blocks, each CTA loading its half
-    of a block's rows as a box of 64 or 128 rows. From 512 rows per expert
-    (T = 2100, 3001) the tiles are 512 tokens wide, two accumulators per
-    weight tile, the second one empty in tiles with at most 256 rows."""
+    of a block's rows as a box of 64 or 128 rows; at T = 2100 and 3001
+    experts have more rows than weight rows and run token block by token
+    block."""
     wl = synth.workload("tiny").with_T(T)
     x, _, wr, b, r = _inputs.routed_inputs(wl)
     g = _gpu.forward(wl, x)
