@@ -3,11 +3,13 @@
 // "Residual Stream": the router is computed in FP32).
 //
 // Stage 0 (router_logits_kernel): logits = x W_r^T on CUDA cores in FP32,
-// 128 tokens x 128 experts per CTA, 8 x 8 per thread, with an optional split
-// over H (at most 16 parts) so that small batches still fill the GPU. Partial
-// sums are written per split and added in split order by stage 1, so the
-// result does not depend on scheduling. The same kernel clears the dispatch
-// bits that stage 1 sets.
+// 128 tokens x 128 experts per CTA, 8 x 8 per thread as paired FP32 FMAs
+// (fma.rn.f32x2), 32 k per shared-memory stage, with an optional split over H
+// (at most 16 parts) so that small batches still fill the GPU. Each logit is
+// a chain of FP32 FMAs in ascending k inside its split; partial sums are
+// written per split and added in split order by stage 1, so the result does
+// not depend on scheduling. The same kernel clears the dispatch bits that
+// stage 1 sets.
 //
 // Stage 1 (router_topk_kernel): one warp per token. Lane l holds PER
 // consecutive experts; a group of E/G experts spans E/G/PER lanes. The warp
@@ -26,17 +28,33 @@ namespace {
 
 constexpr int kRBM = 128;  // tokens per CTA
 constexpr int kRBE = 128;  // experts per CTA
-constexpr int kRBK = 16;   // K per shared-memory stage
+constexpr int kRBK = 32;   // K per shared-memory stage
 constexpr int kMaxSplit = 16;
+constexpr int kRouterSmem = 2 * 2 * kRBK * kRBM * 4;  // [2 stages][x, w][kRBK][128] fp32
 
-__global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
-                                                            const float* __restrict__ wr,
-                                                            float* __restrict__ part, int T, int H,
-                                                            int E, int kc,
-                                                            uint32_t* __restrict__ bits,
-                                                            int64_t n_bits_words) {
-  __shared__ __align__(16) float xs[2][kRBK][kRBM];
-  __shared__ __align__(16) float wsm[2][kRBK][kRBE];
+// d = a * b + c on two FP32 lanes at once (fma.rn.f32x2: each lane is an
+// ordinary round-to-nearest FP32 FMA, so results equal two fmaf calls). Half
+// the FMA instructions of the scalar loop for the same arithmetic.
+__device__ __forceinline__ void fma2(unsigned long long& d, unsigned long long a,
+                                     unsigned long long b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+
+__device__ __forceinline__ unsigned long long splat2(float v) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+  return r;
+}
+
+__global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* __restrict__ x,
+                                                               const float* __restrict__ wr,
+                                                               float* __restrict__ part, int T,
+                                                               int H, int E, int kc,
+                                                               uint32_t* __restrict__ bits,
+                                                               int64_t n_bits_words) {
+  extern __shared__ __align__(16) float rsm[];
+  float (*xs)[kRBK][kRBM] = reinterpret_cast<float (*)[kRBK][kRBM]>(rsm);
+  float (*wsm)[kRBK][kRBE] = reinterpret_cast<float (*)[kRBK][kRBE]>(rsm + 2 * kRBK * kRBM);
   const int tid = threadIdx.x;
   {  // clear the dispatch bits set by stage 1
     const int64_t nthreads = (int64_t)gridDim.x * gridDim.y * gridDim.z * blockDim.x;
@@ -47,43 +65,50 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
   const int kbeg = blockIdx.z * kc;
   // compute mapping: tokens {ty*4+i, 64+ty*4+i}, experts {tx*4+j, 64+tx*4+j}
   const int tx = tid & 15, ty = tid >> 4;
-  // loader mapping: x row tid&127 at k offset (tid>>7)*8; w row tid&127 at (tid>>7)*4 and +8
-  const int lrow = tid & 127, lx_k = (tid >> 7) * 8, lw_k = (tid >> 7) * 4;
+  // loader mapping: row tid&127 (a token of x, an expert of W_r), k offset
+  // (tid>>7)*16 inside the stage: 16 consecutive k of one row per thread
+  const int lrow = tid & 127, lk = (tid >> 7) * 16;
   const bool x_ok = m0 + lrow < T, w_ok = e0 + lrow < E;
   const uint16_t* xrow = x + (size_t)(x_ok ? m0 + lrow : 0) * H;
   const float* wrow = wr + (size_t)(w_ok ? e0 + lrow : 0) * H;
 
-  uint4 xr;
-  float4 wv0, wv1;
+  uint4 xr[2];
+  float4 wv[4];
   auto load = [&](int k0) {
-    xr = x_ok ? __ldg(reinterpret_cast<const uint4*>(xrow + k0 + lx_k)) : make_uint4(0, 0, 0, 0);
-    wv0 = w_ok ? __ldg(reinterpret_cast<const float4*>(wrow + k0 + lw_k))
-               : make_float4(0.f, 0.f, 0.f, 0.f);
-    wv1 = w_ok ? __ldg(reinterpret_cast<const float4*>(wrow + k0 + lw_k + 8))
-               : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      xr[q] = x_ok ? __ldg(reinterpret_cast<const uint4*>(xrow + k0 + lk + 8 * q))
+                   : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      wv[q] = w_ok ? __ldg(reinterpret_cast<const float4*>(wrow + k0 + lk + 4 * q))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
   };
   auto store = [&](int buf) {
-    const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      xs[buf][lx_k + 2 * j][lrow] = __uint_as_float(xw[j] << 16);
-      xs[buf][lx_k + 2 * j + 1][lrow] = __uint_as_float(xw[j] & 0xFFFF0000u);
+    for (int q = 0; q < 2; ++q) {
+      const uint32_t xw[4] = {xr[q].x, xr[q].y, xr[q].z, xr[q].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {  // bf16 -> fp32 is exact: the bits move up 16
+        xs[buf][lk + 8 * q + 2 * j][lrow] = __uint_as_float(xw[j] << 16);
+        xs[buf][lk + 8 * q + 2 * j + 1][lrow] = __uint_as_float(xw[j] & 0xFFFF0000u);
+      }
     }
-    wsm[buf][lw_k + 0][lrow] = wv0.x;
-    wsm[buf][lw_k + 1][lrow] = wv0.y;
-    wsm[buf][lw_k + 2][lrow] = wv0.z;
-    wsm[buf][lw_k + 3][lrow] = wv0.w;
-    wsm[buf][lw_k + 8][lrow] = wv1.x;
-    wsm[buf][lw_k + 9][lrow] = wv1.y;
-    wsm[buf][lw_k + 10][lrow] = wv1.z;
-    wsm[buf][lw_k + 11][lrow] = wv1.w;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      wsm[buf][lk + 4 * q + 0][lrow] = wv[q].x;
+      wsm[buf][lk + 4 * q + 1][lrow] = wv[q].y;
+      wsm[buf][lk + 4 * q + 2][lrow] = wv[q].z;
+      wsm[buf][lk + 4 * q + 3][lrow] = wv[q].w;
+    }
   };
 
-  float acc[8][8];
+  // acc[i][jj] holds experts (2 jj, 2 jj + 1) of this thread's 8 for token i
+  unsigned long long acc[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0ull;
 
   const int nk = kc / kRBK;
   load(kbeg);
@@ -96,14 +121,16 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
     for (int k = 0; k < kRBK; ++k) {
       const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 4]);
       const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][k][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&wsm[buf][k][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&wsm[buf][k][64 + tx * 4]);
+      const ulonglong2 b0 = *reinterpret_cast<const ulonglong2*>(&wsm[buf][k][tx * 4]);
+      const ulonglong2 b1 = *reinterpret_cast<const ulonglong2*>(&wsm[buf][k][64 + tx * 4]);
       const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const unsigned long long bv[4] = {b0.x, b0.y, b1.x, b1.y};
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 8; ++i) {
+        const unsigned long long a2 = splat2(av[i]);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) fma2(acc[i][j], a2, bv[j]);
+      }
     }
     if (it + 1 < nk) store(buf ^ 1);
     __syncthreads();
@@ -116,13 +143,15 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
     if (t >= T) continue;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
+      float v[4];
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(v[0]), "=f"(v[1]) : "l"(acc[i][2 * h]));
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(v[2]), "=f"(v[3]) : "l"(acc[i][2 * h + 1]));
       const int e = e0 + h * 64 + tx * 4;
       if ((E & 3) == 0 && e + 3 < E) {
-        *reinterpret_cast<float4*>(out + (size_t)t * E + e) =
-            make_float4(acc[i][4 * h], acc[i][4 * h + 1], acc[i][4 * h + 2], acc[i][4 * h + 3]);
+        *reinterpret_cast<float4*>(out + (size_t)t * E + e) = make_float4(v[0], v[1], v[2], v[3]);
       } else {
         for (int q = 0; q < 4; ++q)
-          if (e + q < E) out[(size_t)t * E + e + q] = acc[i][4 * h + q];
+          if (e + q < E) out[(size_t)t * E + e + q] = v[q];
       }
     }
   }
@@ -350,9 +379,16 @@ cudaError_t launch_router_logits(const beam_moe_cfg& c, const Layout& L, const u
                                  const float* w_router, char* ws, cudaStream_t st) {
   if (L.router_tc) return launch_router_tc(c, L, x, w_router, ws, st);
   const int H = c.hidden, E = c.n_experts;
+  static PerDevice configured;  // the shared-memory attribute, once per device
+  int unused = 0;
+  cudaError_t err = per_device(configured, &unused, [](int*) {
+    return cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kRouterSmem);
+  });
+  if (err != cudaSuccess) return err;
   dim3 grid((unsigned)((L.T + kRBM - 1) / kRBM), (unsigned)((E + kRBE - 1) / kRBE),
             (unsigned)L.split_k);
-  router_logits_kernel<<<grid, 256, 0, st>>>(
+  router_logits_kernel<<<grid, 256, kRouterSmem, st>>>(
       x, w_router, reinterpret_cast<float*>(ws + L.logits), (int)L.T, H, E, H / L.split_k,
       reinterpret_cast<uint32_t*>(ws + L.chunk_mask), (int64_t)L.nchunks * E * kChunkWords);
   return cudaGetLastError();
