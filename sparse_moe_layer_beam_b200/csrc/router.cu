@@ -46,6 +46,23 @@ __device__ __forceinline__ unsigned long long splat2(float v) {
   return r;
 }
 
+// 4-byte asynchronous copy global -> shared (zero-filled when src_bytes is 0),
+// and the wait for every copy this thread has issued.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* __restrict__ x,
                                                                const float* __restrict__ wr,
                                                                float* __restrict__ part, int T,
@@ -72,19 +89,17 @@ __global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* _
   const uint16_t* xrow = x + (size_t)(x_ok ? m0 + lrow : 0) * H;
   const float* wrow = wr + (size_t)(w_ok ? e0 + lrow : 0) * H;
 
+  // x goes through registers (bf16 -> fp32 on the way into shared memory);
+  // W_r, already fp32, is copied asynchronously straight into its transposed
+  // place, one 4-byte element per copy, so no register holds it.
   uint4 xr[2];
-  float4 wv[4];
-  auto load = [&](int k0) {
+  auto load_x = [&](int k0) {
 #pragma unroll
     for (int q = 0; q < 2; ++q)
       xr[q] = x_ok ? __ldg(reinterpret_cast<const uint4*>(xrow + k0 + lk + 8 * q))
                    : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      wv[q] = w_ok ? __ldg(reinterpret_cast<const float4*>(wrow + k0 + lk + 4 * q))
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
   };
-  auto store = [&](int buf) {
+  auto store_x = [&](int buf) {
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const uint32_t xw[4] = {xr[q].x, xr[q].y, xr[q].z, xr[q].w};
@@ -94,13 +109,12 @@ __global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* _
         xs[buf][lk + 8 * q + 2 * j + 1][lrow] = __uint_as_float(xw[j] & 0xFFFF0000u);
       }
     }
+  };
+  auto copy_w = [&](int k0, int buf) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      wsm[buf][lk + 4 * q + 0][lrow] = wv[q].x;
-      wsm[buf][lk + 4 * q + 1][lrow] = wv[q].y;
-      wsm[buf][lk + 4 * q + 2][lrow] = wv[q].z;
-      wsm[buf][lk + 4 * q + 3][lrow] = wv[q].w;
-    }
+    for (int q = 0; q < 16; ++q)
+      cp_async4(&wsm[buf][lk + q][lrow], wrow + k0 + lk + q, w_ok ? 4u : 0u);
+    cp_async_commit();
   };
 
   // acc[i][jj] holds experts (2 jj, 2 jj + 1) of this thread's 8 for token i
@@ -111,12 +125,17 @@ __global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* _
     for (int j = 0; j < 4; ++j) acc[i][j] = 0ull;
 
   const int nk = kc / kRBK;
-  load(kbeg);
-  store(0);
+  load_x(kbeg);
+  copy_w(kbeg, 0);
+  store_x(0);
+  cp_async_wait_all();
   __syncthreads();
   for (int it = 0; it < nk; ++it) {
     const int buf = it & 1;
-    if (it + 1 < nk) load(kbeg + (it + 1) * kRBK);
+    if (it + 1 < nk) {
+      load_x(kbeg + (it + 1) * kRBK);
+      copy_w(kbeg + (it + 1) * kRBK, buf ^ 1);
+    }
 #pragma unroll
     for (int k = 0; k < kRBK; ++k) {
       const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 4]);
@@ -132,7 +151,10 @@ __global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* _
         for (int j = 0; j < 4; ++j) fma2(acc[i][j], a2, bv[j]);
       }
     }
-    if (it + 1 < nk) store(buf ^ 1);
+    if (it + 1 < nk) {
+      store_x(buf ^ 1);
+      cp_async_wait_all();
+    }
     __syncthreads();
   }
 
