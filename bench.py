@@ -53,32 +53,42 @@ METRIC = "MoE-block tokens/s; achieved TFLOP/s or HBM GB/s as % of B200 roofline
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 STAGES = ("router_gemm", "router_topk", "scan", "permute", "gateup_gemm", "down_gemm", "combine")
-GEMM_SOURCES = ("sparse_moe_layer_beam_b200/csrc/grouped_gemm.cu",
-                "sparse_moe_layer_beam_b200/csrc/grouped_gemm.cuh",
-                "sparse_moe_layer_beam_b200/csrc/sm100.cuh")
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the gate/up
-# kernel per touched expert, from an ncu capture of the same kernel on a small
-# decode-like case; valid only for the decode workload and only while the
-# kernel sources hash to `sources_sha256` (any edit to them voids it).
-GATEUP_TRAFFIC = {"workload": "decode", "bytes_per_touched_expert": 52619897,
-                  "sources_sha256": "d2654dc8e6ea4346cb90aa5c6d956b21c8ca1ae00fcb5da28860253f4dd80d0b"}
+# kernel, from ncu captures of small cases in the same regime as a workload,
+# scaled to a full launch by the unit named: touched experts at decode (the
+# weights dominate; about 2 rows per expert in both), assignments for the long
+# chunk (2048 rows per expert in both). A record is valid only while the
+# sources of the kernel that runs hash to `sha256`; any edit voids it.
+GATEUP_TRAFFIC = {
+    "decode": {"per": "touched_expert", "bytes": None,
+               "sources": ("sparse_moe_layer_beam_b200/csrc/grouped_gemm.cu",
+                           "sparse_moe_layer_beam_b200/csrc/grouped_gemm.cuh",
+                           "sparse_moe_layer_beam_b200/csrc/sm100.cuh"),
+               "sha256": None},
+    "long": {"per": "assignment", "bytes": None,
+             "sources": ("sparse_moe_layer_beam_b200/csrc/grouped_gemm_2sm.cu",
+                         "sparse_moe_layer_beam_b200/csrc/grouped_gemm.cuh",
+                         "sparse_moe_layer_beam_b200/csrc/sm100.cuh"),
+             "sha256": None},
+}
 
 
-def gemm_sources_sha256():
+def sources_sha256(paths):
     import hashlib
     h = hashlib.sha256()
-    for rel in GEMM_SOURCES:
+    for rel in paths:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def gateup_traffic(wl, touched):
-    rec = GATEUP_TRAFFIC
-    if (rec["bytes_per_touched_expert"] is None or wl.name != rec["workload"]
-            or gemm_sources_sha256() != rec["sources_sha256"]):
+def gateup_traffic(wl, alg):
+    """Estimated DRAM bytes of one gate/up launch, or None without a valid record."""
+    rec = GATEUP_TRAFFIC.get(wl.name)
+    if rec is None or rec["bytes"] is None or sources_sha256(rec["sources"]) != rec["sha256"]:
         return None
-    return rec["bytes_per_touched_expert"] * touched
+    units = alg["touched_experts"] if rec["per"] == "touched_expert" else wl.T * wl.K
+    return rec["bytes"] * units
 
 
 def host_chunking(T, nvfp4):
@@ -476,7 +486,7 @@ def measure(args, wl, ex, dev, stream, rank, world, local):
     roof, block = roofline(alg, None if args.replay else gate_ms, ms_step, peaks, peak_kind,
                            nvfp4)
     # the recorded DRAM traffic belongs to the bf16 gate/up kernel only
-    roof["traffic"] = None if nvfp4 else gateup_traffic(wl, alg["touched_experts"])
+    roof["traffic"] = None if nvfp4 else gateup_traffic(wl, alg)
     # router GEMM (plus the weight split on tensor cores), top-k, scan,
     # permute, gate/up, down, combine; replayed routes: the route copy, scan,
     # permute, gate/up, down, combine

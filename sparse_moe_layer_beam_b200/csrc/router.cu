@@ -30,7 +30,9 @@ constexpr int kRBM = 128;  // tokens per CTA
 constexpr int kRBE = 128;  // experts per CTA
 constexpr int kRBK = 32;   // K per shared-memory stage
 constexpr int kMaxSplit = 16;
-constexpr int kRouterSmem = 2 * 2 * kRBK * kRBM * 4;  // [2 stages][x, w][kRBK][128] fp32
+constexpr int kRawLd = kRBK + 4;  // row stride of the raw W_r stage (16-byte chunks spread over banks)
+// [2 stages][x, w][kRBK][128] fp32, then the raw W_r stage [128][kRawLd] fp32
+constexpr int kRouterSmem = (2 * 2 * kRBK * kRBM + kRBE * kRawLd) * 4;
 
 // d = a * b + c on two FP32 lanes at once (fma.rn.f32x2: each lane is an
 // ordinary round-to-nearest FP32 FMA, so results equal two fmaf calls). Half
@@ -46,21 +48,21 @@ __device__ __forceinline__ unsigned long long splat2(float v) {
   return r;
 }
 
-// 4-byte asynchronous copy global -> shared (zero-filled when src_bytes is 0),
-// and the wait for every copy this thread has issued.
-__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(
+// 16-byte asynchronous copy global -> shared (zero-filled when src_bytes is
+// 0), and the wait for every copy this thread has issued.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
                    static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
                "l"(src), "r"(src_bytes)
                : "memory");
 }
 
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 __global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* __restrict__ x,
@@ -72,6 +74,7 @@ __global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* _
   extern __shared__ __align__(16) float rsm[];
   float (*xs)[kRBK][kRBM] = reinterpret_cast<float (*)[kRBK][kRBM]>(rsm);
   float (*wsm)[kRBK][kRBE] = reinterpret_cast<float (*)[kRBK][kRBE]>(rsm + 2 * kRBK * kRBM);
+  float (*raw)[kRawLd] = reinterpret_cast<float (*)[kRawLd]>(rsm + 4 * kRBK * kRBM);
   const int tid = threadIdx.x;
   {  // clear the dispatch bits set by stage 1
     const int64_t nthreads = (int64_t)gridDim.x * gridDim.y * gridDim.z * blockDim.x;
@@ -89,9 +92,10 @@ __global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* _
   const uint16_t* xrow = x + (size_t)(x_ok ? m0 + lrow : 0) * H;
   const float* wrow = wr + (size_t)(w_ok ? e0 + lrow : 0) * H;
 
-  // x goes through registers (bf16 -> fp32 on the way into shared memory);
-  // W_r, already fp32, is copied asynchronously straight into its transposed
-  // place, one 4-byte element per copy, so no register holds it.
+  // x goes through registers (bf16 -> fp32 on the way into shared memory).
+  // W_r, already fp32, is copied asynchronously one stage ahead into a raw
+  // row-major stage; each thread then moves the cells it copied itself into
+  // their transposed place, so no register holds W_r across the compute.
   uint4 xr[2];
   auto load_x = [&](int k0) {
 #pragma unroll
@@ -110,11 +114,22 @@ __global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* _
       }
     }
   };
-  auto copy_w = [&](int k0, int buf) {
+  auto copy_w = [&](int k0) {
 #pragma unroll
-    for (int q = 0; q < 16; ++q)
-      cp_async4(&wsm[buf][lk + q][lrow], wrow + k0 + lk + q, w_ok ? 4u : 0u);
+    for (int q = 0; q < 4; ++q)
+      cp_async16(&raw[lrow][lk + 4 * q], wrow + k0 + lk + 4 * q, w_ok ? 16u : 0u);
     cp_async_commit();
+  };
+  auto store_w = [&](int buf) {
+    cp_async_wait_all();  // this thread's own copies: no barrier needed to read them
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = *reinterpret_cast<const float4*>(&raw[lrow][lk + 4 * q]);
+      wsm[buf][lk + 4 * q + 0][lrow] = v.x;
+      wsm[buf][lk + 4 * q + 1][lrow] = v.y;
+      wsm[buf][lk + 4 * q + 2][lrow] = v.z;
+      wsm[buf][lk + 4 * q + 3][lrow] = v.w;
+    }
   };
 
   // acc[i][jj] holds experts (2 jj, 2 jj + 1) of this thread's 8 for token i
@@ -126,15 +141,15 @@ __global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* _
 
   const int nk = kc / kRBK;
   load_x(kbeg);
-  copy_w(kbeg, 0);
+  copy_w(kbeg);
   store_x(0);
-  cp_async_wait_all();
+  store_w(0);
   __syncthreads();
   for (int it = 0; it < nk; ++it) {
     const int buf = it & 1;
     if (it + 1 < nk) {
       load_x(kbeg + (it + 1) * kRBK);
-      copy_w(kbeg + (it + 1) * kRBK, buf ^ 1);
+      copy_w(kbeg + (it + 1) * kRBK);
     }
 #pragma unroll
     for (int k = 0; k < kRBK; ++k) {
@@ -153,7 +168,7 @@ __global__ void __launch_bounds__(256, 2) router_logits_kernel(const uint16_t* _
     }
     if (it + 1 < nk) {
       store_x(buf ^ 1);
-      cp_async_wait_all();
+      store_w(buf ^ 1);
     }
     __syncthreads();
   }

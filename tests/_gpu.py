@@ -255,23 +255,44 @@ def oracle_hidden(wl, x_bits, tokens, r_oracle):
     return oracle.hidden(cfg, x_bits[np.asarray(tokens)], ids, w13)
 
 
-# NVFP4 outputs, beyond their own bf16 rounding: max |err| - half a bf16 step
-# of the output <= TOL_NVFP4 x RMS. The block's tolerance of 2e-2 x RMS is
-# stated for BF16 weights and activations; NVFP4 outputs have heavier tails
-# (RMS about 1.75, elements up to about 20 at Beam's shapes), where half a
-# bf16 step alone (1/32 in [8, 16), 1/16 in [16, 32)) exceeds 2e-2 x RMS. The
-# rest of the NVFP4 arithmetic (x and h quantised by the same rule on both
-# sides, FP32 against fp64 sums) is held to 1e-2 x RMS.
-TOL_NVFP4 = 1e-2
+# NVFP4 outputs. The block's tolerance of 2e-2 x RMS is stated for BF16 weights
+# and activations; for NVFP4 it is derived from the arithmetic:
+# - each element may differ by half a bf16 step of the output (its one
+#   rounding; NVFP4 outputs have heavier tails, RMS about 1.75 and elements up
+#   to about 20 at Beam's shapes, where half a step reaches 1/16) plus
+#   TOL_NVFP4_ELEM x RMS: where the GPU's FP32 sums and the oracle's fp64 sums
+#   put an element of h on either side of an E2M1 decision boundary, its code
+#   differs by one step (up to twice the block scale, about amax / 3), which
+#   moves out[j] by w_k W2[j, i] times that: up to about 0.035 = 0.02 x RMS at
+#   Beam's shapes (w_k about 0.3, |W2| <= 0.088 for the synthetic experts,
+#   block amax about 4), a few times per thousand rows;
+# - the RMS of the error over all compared elements may exceed that of the
+#   output's own bf16 rounding by at most TOL_NVFP4_RMS x RMS, which isolated
+#   flips cannot reach but any systematic error (a scale, a code table, a
+#   dropped term) would.
+TOL_NVFP4_ELEM = 3e-2
+TOL_NVFP4_RMS = 1e-3
 
 
-def nvfp4_excess(out_bits, ref):
-    """(max over elements of (|err| - half a bf16 step at the output) / RMS, RMS)."""
+def nvfp4_errors(out_bits, ref):
+    """(max over elements of (|err| - half a bf16 step at the output) / RMS,
+    (RMS of the error - RMS of rounding ref to bf16) / RMS, RMS)."""
     got = synth.bf16_to_f32(out_bits).astype(np.float64)
     rms = np.sqrt(np.mean(ref ** 2))
     _, e = np.frexp(np.maximum(np.abs(ref), np.abs(got)))
     half_step = np.ldexp(1.0, e - 9)  # bf16 keeps 8 significant bits
-    return ((np.abs(got - ref) - half_step) / rms).max(), rms
+    excess = ((np.abs(got - ref) - half_step) / rms).max()
+    m, ex = np.frexp(ref)
+    rounded = np.ldexp(np.round(m * 256.0), ex - 8)  # ref to bf16, ties to even
+    rms_err = np.sqrt(np.mean((got - ref) ** 2))
+    rms_round = np.sqrt(np.mean((rounded - ref) ** 2))
+    return excess, (rms_err - rms_round) / rms, rms
+
+
+def check_nvfp4(out_bits, ref):
+    excess, rms_excess, rms = nvfp4_errors(out_bits, ref)
+    assert excess <= TOL_NVFP4_ELEM, (excess, rms)
+    assert rms_excess <= TOL_NVFP4_RMS, (rms_excess, rms)
 
 
 def max_rel_err(out_bits, ref):

@@ -50,3 +50,20 @@ def test_no_kernel_time_gives_no_fraction_and_fallback_is_named():
     assert roof["achieved"] is None and roof["frac"] is None
     assert roof["peak_source"] == "fallback"
     assert block["hbm_frac"] > 0
+
+
+def test_gateup_traffic_scales_by_its_unit_and_needs_matching_sources(monkeypatch):
+    import synth
+
+    rec = dict(bench.GATEUP_TRAFFIC["long"], bytes=100, sha256="not-the-sources")
+    monkeypatch.setitem(bench.GATEUP_TRAFFIC, "long", rec)
+    wl = synth.workload("long")
+    alg = {"touched_experts": 3}
+    assert bench.gateup_traffic(wl, alg) is None  # sources changed since the capture
+    rec["sha256"] = bench.sources_sha256(rec["sources"])
+    assert bench.gateup_traffic(wl, alg) == 100 * wl.T * wl.K  # per assignment
+    dec = dict(bench.GATEUP_TRAFFIC["decode"], bytes=7)
+    dec["sha256"] = bench.sources_sha256(dec["sources"])
+    monkeypatch.setitem(bench.GATEUP_TRAFFIC, "decode", dec)
+    assert bench.gateup_traffic(synth.workload("decode"), alg) == 21  # per touched expert
+    assert bench.gateup_traffic(synth.workload("prefill"), alg) is None  # no record

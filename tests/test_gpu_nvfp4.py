@@ -2,7 +2,8 @@
 exactly, values exactly), the device weight fill against the host generator,
 and the whole block (routing bit-exact; outputs against the oracle's fp64
 evaluation on exactly dequantised values within half a bf16 step of the
-output plus 1e-2 x RMS, see _gpu.TOL_NVFP4)."""
+output plus 3e-2 x RMS per element, and an RMS error within 1e-3 x RMS of the
+output's own bf16 rounding: see _gpu.TOL_NVFP4_ELEM for the derivation)."""
 import numpy as np
 import pytest
 import torch
@@ -56,8 +57,7 @@ def test_nvfp4_forward_tiny(T):
     _gpu.check_routes(g, r, wl.E)
     tokens = np.arange(wl.T) if wl.T <= 256 else synth.sample_tokens(wl.T, 64)
     ref = _gpu.oracle_outputs_nvfp4(wl, x, tokens, r, batch=64)
-    err, rms = _gpu.nvfp4_excess(g["out"][tokens], ref)
-    assert err <= _gpu.TOL_NVFP4, (err, rms)
+    _gpu.check_nvfp4(g["out"][tokens], ref)
 
 
 def _full_case(name, tokens=None):
@@ -73,8 +73,7 @@ def _full_case(name, tokens=None):
     if tokens is None:
         tokens = _gpu.block_cover_tokens(r["ids"], wl.E, 128)
     ref = _gpu.oracle_outputs_nvfp4(wl, x, tokens, r)
-    err, rms = _gpu.nvfp4_excess(g["out"][tokens], ref)
-    assert err <= _gpu.TOL_NVFP4, (err, rms)
+    _gpu.check_nvfp4(g["out"][tokens], ref)
 
 
 def test_nvfp4_decode_full_size():
