@@ -60,16 +60,16 @@ STAGES = ("router_gemm", "router_topk", "scan", "permute", "gateup_gemm", "down_
 # chunk (2048 rows per expert in both). A record is valid only while the
 # sources of the kernel that runs hash to `sha256`; any edit voids it.
 GATEUP_TRAFFIC = {
-    "decode": {"per": "touched_expert", "bytes": None,
+    "decode": {"per": "touched_expert", "bytes": 52566680,
                "sources": ("sparse_moe_layer_beam_b200/csrc/grouped_gemm.cu",
                            "sparse_moe_layer_beam_b200/csrc/grouped_gemm.cuh",
                            "sparse_moe_layer_beam_b200/csrc/sm100.cuh"),
-               "sha256": None},
-    "long": {"per": "assignment", "bytes": None,
+               "sha256": "060a094ff9b43d310b473a3d5a36f143d5e4194019bac328c9f6826727246051"},
+    "long": {"per": "assignment", "bytes": 69702,
              "sources": ("sparse_moe_layer_beam_b200/csrc/grouped_gemm_2sm.cu",
                          "sparse_moe_layer_beam_b200/csrc/grouped_gemm.cuh",
                          "sparse_moe_layer_beam_b200/csrc/sm100.cuh"),
-             "sha256": None},
+             "sha256": "7b2a4247761de860b02dd0ea5ab0b9e9ccba187200e95c5d012312798e844f8f"},
 }
 
 
