@@ -276,11 +276,8 @@ BEAM_MOE_API beam_moe_status beam_moe_nvfp4_quantize(int64_t rows, int64_t K, co
  *   pos     [T][K] int32       permuted row of each (token, slot): the rows of
  *                              an expert are contiguous from offsets[e], in
  *                              ascending token order
- *   tok     [T*K] int32        token of each permuted row (the inverse of pos)
  *   xp      [T*K][H] bf16      permuted token rows (valid after stage 3 and
- *                              until stage 5 overwrites them with y), written
- *                              only when gather is 0: with gather = 1 the
- *                              gate/up GEMM reads each row straight from x
+ *                              until stage 5 overwrites them with y)
  *   h       [T*K][I] bf16      silu(g) * u of each permuted row (after stage 4)
  *   y       [T*K][H] fp32      down projection of each permuted row (after
  *                              stage 5; the same bytes as xp)
@@ -288,13 +285,11 @@ BEAM_MOE_API beam_moe_status beam_moe_nvfp4_quantize(int64_t rows, int64_t K, co
  * BEAM_MOE_OP_FORWARD. These calls exist for tests and debugging.
  */
 typedef struct beam_moe_ws_layout {
-  int64_t counts, offsets, ids, w, pos, tok, xp, h, y; /* byte offsets in ws    */
+  int64_t counts, offsets, ids, w, pos, xp, h, y; /* byte offsets in ws         */
   int32_t router_splits; /* slices of H whose FP32 partial logits are added  */
   int32_t router_tc;     /* 1: the router GEMM runs on tensor cores           */
   int32_t pair_gateup;   /* 1: gate/up grouped GEMM on CTA pairs              */
   int32_t pair_down;     /* 1: down grouped GEMM on CTA pairs                 */
-  int32_t gather;        /* 1: gate/up reads token rows straight from x; xp is
-                            not written                                       */
 } beam_moe_ws_layout;
 BEAM_MOE_API beam_moe_status beam_moe_workspace_layout(const beam_moe_cfg* cfg, int64_t T,
                                                        beam_moe_op op,

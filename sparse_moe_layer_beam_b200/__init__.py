@@ -53,11 +53,10 @@ class BeamMoeCfg(ctypes.Structure):
 class BeamMoeWsLayout(ctypes.Structure):
     """Byte offsets of the intermediates inside a forward workspace."""
     _fields_ = [("counts", ctypes.c_int64), ("offsets", ctypes.c_int64), ("ids", ctypes.c_int64),
-                ("w", ctypes.c_int64), ("pos", ctypes.c_int64), ("tok", ctypes.c_int64),
-                ("xp", ctypes.c_int64),
+                ("w", ctypes.c_int64), ("pos", ctypes.c_int64), ("xp", ctypes.c_int64),
                 ("h", ctypes.c_int64), ("y", ctypes.c_int64), ("router_splits", ctypes.c_int32),
                 ("router_tc", ctypes.c_int32), ("pair_gateup", ctypes.c_int32),
-                ("pair_down", ctypes.c_int32), ("gather", ctypes.c_int32)]
+                ("pair_down", ctypes.c_int32)]
 
 
 class BeamMoeNvfp4Experts(ctypes.Structure):

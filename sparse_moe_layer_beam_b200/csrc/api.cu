@@ -68,9 +68,6 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool allow_tc) {
   const bool pair_ok = L.bn == 256 && pair_gemm_supported(c);
   L.pair_gateup = (pair_ok && mean_rows >= 64.0) ? 1 : 0;
   L.pair_down = (pair_ok && mean_rows >= 64.0) ? 1 : 0;
-  // The pair gate/up GEMM reads each token's row straight from x (TMA
-  // gather4), so the permute writes no rows for it.
-  L.gather = L.pair_gateup;
 
   size_t o = 0;
   auto take = [&](size_t bytes, size_t align) {
@@ -87,7 +84,6 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool allow_tc) {
   L.ids = take(sizeof(int32_t) * (size_t)L.A, 256);
   L.w = take(sizeof(float) * (size_t)L.A, 256);
   L.pos = take(sizeof(int32_t) * (size_t)L.A, 256);
-  L.tok = take(sizeof(int32_t) * (size_t)L.A, 256);
   L.chunk_cnt = take(sizeof(int32_t) * (size_t)L.nchunks * E, 256);
   L.chunk_mask = take(sizeof(uint32_t) * (size_t)L.nchunks * E * kChunkWords, 256);
   L.logits = take(sizeof(float) * (size_t)L.split_k * T * E, 256);
@@ -293,7 +289,7 @@ beam_moe_status expert_path(const beam_moe_cfg* cfg, const Layout& L, const uint
   BEAM_CUDA(beam::launch_permute(*cfg, L, x, ws, st));
   BEAM_CUDA(rec.mark(4));
   if (last < 4) return BEAM_MOE_OK;
-  BEAM_CUDA(L.pair_gateup ? beam::launch_gateup_pair(*cfg, L, w13, ws, st, x)
+  BEAM_CUDA(L.pair_gateup ? beam::launch_gateup_pair(*cfg, L, w13, ws, st)
                           : beam::launch_gateup(*cfg, L, w13, ws, st));
   BEAM_CUDA(rec.mark(5));
   if (last < 5) return BEAM_MOE_OK;
@@ -653,8 +649,6 @@ beam_moe_status beam_moe_workspace_layout(const beam_moe_cfg* cfg, int64_t T, be
   out->ids = (int64_t)L.ids;
   out->w = (int64_t)L.w;
   out->pos = (int64_t)L.pos;
-  out->tok = (int64_t)L.tok;
-  out->gather = L.gather;
   out->xp = (int64_t)L.xp;
   out->h = (int64_t)L.h;
   out->y = (int64_t)L.xp;
@@ -764,7 +758,7 @@ beam_moe_status ep_checks(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep) {
 // its status word is the workspace's first (shared with the expert stage).
 Layout ep_routing(const beam_moe_cfg& c, int64_t T, int sms, size_t base) {
   Layout L = beam::make_layout(c, T, sms);
-  size_t* f[] = {&L.counts, &L.offsets, &L.nb_off, &L.nb2_off, &L.ids, &L.w, &L.pos, &L.tok,
+  size_t* f[] = {&L.counts, &L.offsets, &L.nb_off, &L.nb2_off, &L.ids, &L.w, &L.pos,
                  &L.chunk_cnt, &L.chunk_mask, &L.logits, &L.w3, &L.route_end, &L.xp, &L.h,
                  &L.total};
   for (size_t* v : f) *v += base;

@@ -111,53 +111,28 @@ __global__ void __launch_bounds__(1024) scan_kernel(const uint32_t* __restrict__
   }
 }
 
-// Permuted row of assignment (t, e): the expert's first row in t's chunk plus
-// the number of earlier tokens of the chunk routed to e; -1 for a dropped id.
-__device__ __forceinline__ int row_of(int t, int e, int E, const int32_t* __restrict__ chunk_base,
-                                      const uint32_t* __restrict__ chunk_mask) {
-  if (e < 0 || e >= E) return -1;
-  const int c = t / kChunk, tl = t - c * kChunk;
-  const uint32_t* m = chunk_mask + ((size_t)c * E + e) * kChunkWords;
-  int rank = 0;
-  for (int wd = 0; wd < (tl >> 5); ++wd) rank += __popc(m[wd]);
-  rank += __popc(m[tl >> 5] & ((1u << (tl & 31)) - 1u));
-  return chunk_base[(size_t)c * E + e] + rank;
-}
-
-// Positions only, one thread per assignment: pos[t][k] and tok[row] = t.
-// Used when the gate/up GEMM gathers the token rows from x itself.
-__global__ void __launch_bounds__(256) positions_kernel(int64_t A, int K, int E,
-                                                        const int32_t* __restrict__ ids,
-                                                        const int32_t* __restrict__ chunk_base,
-                                                        const uint32_t* __restrict__ chunk_mask,
-                                                        int32_t* __restrict__ pos,
-                                                        int32_t* __restrict__ tok) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= A) return;
-  const int t = (int)(i / K);
-  const int p = row_of(t, ids[i], E, chunk_base, chunk_mask);
-  pos[i] = p;
-  if (p >= 0) tok[p] = t;
-}
-
-// Positions, tok[row] = t, and x[t] copied to each of its K rows.
 __global__ void __launch_bounds__(128) permute_kernel(const uint16_t* __restrict__ x, int H, int K,
                                                       int E, const int32_t* __restrict__ ids,
                                                       const int32_t* __restrict__ chunk_base,
                                                       const uint32_t* __restrict__ chunk_mask,
                                                       int32_t* __restrict__ pos,
-                                                      int32_t* __restrict__ tok,
                                                       uint16_t* __restrict__ xp) {
   __shared__ int s_pos[32];
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
   if (tid < K) {
-    const int p = row_of(t, ids[(size_t)t * K + tid], E, chunk_base, chunk_mask);
-    s_pos[tid] = p;
-    if (blockIdx.y == 0) {
-      pos[(size_t)t * K + tid] = p;
-      if (p >= 0) tok[p] = t;
+    const int e = ids[(size_t)t * K + tid];
+    int p = -1;
+    if (e >= 0 && e < E) {
+      const int c = t / kChunk, tl = t - c * kChunk;
+      const uint32_t* m = chunk_mask + ((size_t)c * E + e) * kChunkWords;
+      int rank = 0;
+      for (int wd = 0; wd < (tl >> 5); ++wd) rank += __popc(m[wd]);
+      rank += __popc(m[tl >> 5] & ((1u << (tl & 31)) - 1u));
+      p = chunk_base[(size_t)c * E + e] + rank;
     }
+    s_pos[tid] = p;
+    if (blockIdx.y == 0) pos[(size_t)t * K + tid] = p;
   }
   __syncthreads();
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
@@ -223,19 +198,11 @@ cudaError_t launch_scan(const beam_moe_cfg& c, const Layout& L, char* ws, int32_
 
 cudaError_t launch_permute(const beam_moe_cfg& c, const Layout& L, const uint16_t* x, char* ws,
                            cudaStream_t st) {
-  if (L.gather) {
-    positions_kernel<<<(unsigned)((L.A + 255) / 256), 256, 0, st>>>(
-        L.A, c.top_k, c.n_experts, reinterpret_cast<const int32_t*>(ws + L.ids),
-        reinterpret_cast<const int32_t*>(ws + L.chunk_cnt),
-        reinterpret_cast<const uint32_t*>(ws + L.chunk_mask),
-        reinterpret_cast<int32_t*>(ws + L.pos), reinterpret_cast<int32_t*>(ws + L.tok));
-    return cudaGetLastError();
-  }
   permute_kernel<<<dim3((unsigned)L.T, (unsigned)h_slices(L.T, c.hidden / 8)), 128, 0, st>>>(
       x, c.hidden, c.top_k, c.n_experts, reinterpret_cast<const int32_t*>(ws + L.ids),
       reinterpret_cast<const int32_t*>(ws + L.chunk_cnt),
       reinterpret_cast<const uint32_t*>(ws + L.chunk_mask), reinterpret_cast<int32_t*>(ws + L.pos),
-      reinterpret_cast<int32_t*>(ws + L.tok), reinterpret_cast<uint16_t*>(ws + L.xp));
+      reinterpret_cast<uint16_t*>(ws + L.xp));
   return cudaGetLastError();
 }
 

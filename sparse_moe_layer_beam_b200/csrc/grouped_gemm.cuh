@@ -20,9 +20,6 @@ struct GemmParams {
   int up_rows;  // row offset of the up projection inside an expert (I)
   int n_mblk;   // 128-row weight blocks per expert (I / 128 or H / 128)
   unsigned* status;
-  const int32_t* tok;  // [rows] token of each permuted row (gathered gate/up only)
-  int64_t rows;        // permuted rows (A)
-  int64_t tokens;      // rows of x (T; gathered gate/up only)
 };
 
 __host__ __device__ constexpr int pow2_at_least(int v) {

@@ -81,10 +81,7 @@ struct PairCfg {
 
 // EPRET: the down GEMM under expert parallelism, storing y rows to their
 // source ranks (a separate instance, so that the plain epilogue stays lean).
-// GATHER: gate/up reads each token row straight from x (p.tok names the token
-// of every permuted row): the whole of warp 0 produces, lane 0 arming the
-// stage and loading the weights, every lane gathering four token rows.
-template <bool GATEUP, bool EPRET, bool GATHER = false>
+template <bool GATEUP, bool EPRET>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
                              const __grid_constant__ CUtensorMap tm_x,
@@ -134,74 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_holder;
   const int total = __ldg(p.nb_off + p.E) * p.n_mblk;
 
-  if (GATHER && warp == 0) {
-    // ------------------------------------------- TMA producer (whole warp)
-    const uint64_t pol_stream = policy_evict_first();
-    const uint64_t pol_keep = policy_evict_normal();
-    int stage = 0;
-    uint32_t phase = 0;
-    int64_t issued = 0;
-    for (int tile = pair; tile < total; tile += n_pairs) {
-      int e, mb, nb;
-      decode_pair_tile(tile, p, e, mb, nb);
-      const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
-      const int half = ((rows + 15) & ~15) >> 1;  // 8 .. 128
-      const int64_t r0 = (int64_t)__ldg(p.offsets + e) + nb * kPairN + (int)rank * half;
-      const bool box64 = half <= 64;
-      const uint32_t stage_tx = 2u * (uint32_t)(C::kABytes + (box64 ? 64 : 128) * C::kRowBytes);
-      const int nblk = __ldg(p.nb_off + e + 1) - __ldg(p.nb_off + e);
-      const uint64_t pol_w = nblk == 1 ? pol_stream : pol_keep;
-      const int w0 = mb * 128 + (int)rank * 64;
-      // this lane's four rows of the box: rows past the last routed one
-      // repeat it (the MMA never uses rows past the tile's own), and every
-      // token index is kept inside x
-      const bool mine = 4 * lane < (box64 ? 64 : 128);
-      const int64_t r_last = min((int64_t)__ldg(p.offsets + p.E), p.rows) - 1;
-      int32_t ix[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int64_t r = min(r0 + 4 * lane + j, r_last);
-        const int32_t t = mine ? __ldg(p.tok + r) : 0;
-        ix[j] = (t >= 0 && t < p.tokens) ? t : 0;
-      }
-      bool ok = true;
-      for (int kb = 0; kb < p.nk; ++kb) {
-        int go = 1;
-        uint8_t* sa = smem + stage * C::kStageBytes;
-        const uint32_t bar = mapa_shared(smem_addr(&full[stage]), 0);
-        const int kx = kb * kTileK;
-        if (lane == 0) {
-          go = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, kFlagProducer);
-          if (go) {
-            if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx);
-            tma_load_5d_pair(sa, &tm_w, bar, kx, 0, 0, w0 / 16, e, pol_w);
-          }
-        }
-        if (!__shfl_sync(0xffffffffu, go, 0)) {
-          ok = false;
-          break;
-        }
-        if (mine)
-          tma_gather4_pair(sa + C::kABytes + lane * 4 * C::kRowBytes, &tm_x, bar, kx, ix[0],
-                           ix[1], ix[2], ix[3], pol_keep);
-        ++issued;
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-      if (!ok) break;
-    }
-    // The even CTA's full barriers count both CTAs' copies: wait for the last
-    // ones to land before either CTA can leave.
-    if (leader && lane == 0) {
-      const int64_t first = issued > STAGES ? issued - STAGES : 0;
-      for (int64_t i = first; i < issued; ++i)
-        mbar_wait(&full[i % STAGES], (uint32_t)((i / STAGES) & 1), nullptr, nullptr, 0u,
-                  100000000ull);
-    }
-    __syncwarp();
-  } else if (warp == 0) {
+  if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------ TMA producer
       const uint64_t pol_stream = policy_evict_first();
@@ -386,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool GATEUP, bool EPRET, bool GATHER = false>
+template <bool GATEUP, bool EPRET>
 cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& tx64,
                      const GemmParams& p, const EpReturn& ret, cudaStream_t st) {
   // Per device: the shared-memory attribute and the number of CTA pairs that
@@ -406,14 +336,13 @@ cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const CUtenso
   cfg.numAttrs = 1;
   int resident_pairs = 0;
   cudaError_t err = per_device(pairs, &resident_pairs, [&cfg](int* v) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATEUP, EPRET, GATHER>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATEUP, EPRET>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t probe = cfg;
     probe.gridDim = dim3((unsigned)(device_sm_count() & ~1));
     int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<GATEUP, EPRET, GATHER>,
-                                       &probe);
+    e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<GATEUP, EPRET>, &probe);
     if (e != cudaSuccess) return e;
     if (clusters < 1) return cudaErrorInvalidConfiguration;
     *v = clusters < device_sm_count() / 2 ? clusters : device_sm_count() / 2;
@@ -421,8 +350,7 @@ cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const CUtenso
   });
   if (err != cudaSuccess) return err;
   cfg.gridDim = dim3((unsigned)(2 * resident_pairs));
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATEUP, EPRET, GATHER>, tw, tx, tx64, p,
-                            ret);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATEUP, EPRET>, tw, tx, tx64, p, ret);
 }
 
 // Token-row boxes of 128 and 64 rows over the same matrix.
@@ -435,7 +363,6 @@ cudaError_t encode_xmaps(CUtensorMap* m128, CUtensorMap* m64, const void* base, 
 
 GemmParams base_params(const beam_moe_cfg& c, const Layout& L, char* ws) {
   GemmParams p;
-  memset(&p, 0, sizeof(p));
   p.counts = reinterpret_cast<const int32_t*>(ws + L.counts);
   p.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
   p.nb_off = reinterpret_cast<const int32_t*>(ws + L.nb_off);
@@ -451,18 +378,12 @@ bool pair_gemm_supported(const beam_moe_cfg& c) {
 }
 
 cudaError_t launch_gateup_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w13,
-                               char* ws, cudaStream_t st, const uint16_t* x) {
+                               char* ws, cudaStream_t st) {
   const int H = c.hidden, I = c.inter, E = c.n_experts;
-  const bool gather = L.gather && x;
   CUtensorMap tw, tx, tx64;
   cudaError_t err = encode_tmap_w13_interleaved(&tw, w13, (uint64_t)H, (uint64_t)I, (uint64_t)E);
   if (err != cudaSuccess) return err;
-  if (gather) {  // rows of x, one row high: gathered four at a time
-    err = encode_tmap_2d_bf16(&tx, x, (uint64_t)H, (uint64_t)L.T, kTileK, 1);
-    tx64 = tx;
-  } else {
-    err = encode_xmaps(&tx, &tx64, ws + L.xp, (uint64_t)H, (uint64_t)L.A);
-  }
+  err = encode_xmaps(&tx, &tx64, ws + L.xp, (uint64_t)H, (uint64_t)L.A);
   if (err != cudaSuccess) return err;
   GemmParams p = base_params(c, L, ws);
   p.out = ws + L.h;
@@ -471,12 +392,8 @@ cudaError_t launch_gateup_pair(const beam_moe_cfg& c, const Layout& L, const uin
   p.w_rows = 2 * I;
   p.up_rows = I;
   p.n_mblk = I / 128;  // 128 intermediate indices (gate + up) per pair tile
-  p.tok = reinterpret_cast<const int32_t*>(ws + L.tok);
-  p.rows = L.A;
-  p.tokens = L.T;
   EpReturn none;
   memset(&none, 0, sizeof(none));
-  if (gather) return run_pair<true, false, true>(tw, tx, tx64, p, none, st);
   return run_pair<true, false>(tw, tx, tx64, p, none, st);
 }
 

@@ -78,8 +78,6 @@ struct Layout {
   int bn;           // token tile of the grouped GEMMs
   int pair_gateup; // 1: gate/up grouped GEMM on CTA pairs
   int pair_down;   // 1: down grouped GEMM on CTA pairs
-  int gather;      // 1: the pair gate/up GEMM gathers token rows from x by
-                   // `tok` (TMA gather4); the permute writes positions only
   size_t status;    // uint32[64]
   size_t counts;    // int32[E]
   size_t offsets;   // int32[E + 1] first row of each expert in the permuted rows
@@ -88,7 +86,6 @@ struct Layout {
   size_t ids;       // int32[T * K]
   size_t w;         // float[T * K]
   size_t pos;       // int32[T * K] permuted row of each assignment
-  size_t tok;       // int32[T * K] token of each permuted row
   size_t chunk_cnt; // int32[nchunks * E] first row of each (chunk, expert)
   size_t chunk_mask;// uint32[nchunks * E * kChunkWords]
   size_t logits;    // float[split_k * T * E] partial router logits
@@ -177,10 +174,8 @@ cudaError_t launch_gateup(const beam_moe_cfg& c, const Layout& L, const uint16_t
 cudaError_t launch_down(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2, char* ws,
                         cudaStream_t st);
 bool pair_gemm_supported(const beam_moe_cfg& c);
-// x: the block's input rows; read straight from x (TMA gather4 by L.tok)
-// when L.gather, else the permuted rows in the workspace are read.
 cudaError_t launch_gateup_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w13,
-                               char* ws, cudaStream_t st, const uint16_t* x = nullptr);
+                               char* ws, cudaStream_t st);
 cudaError_t launch_down_pair(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2,
                              char* ws, cudaStream_t st, const EpReturn* ret = nullptr);
 cudaError_t launch_combine(const beam_moe_cfg& c, const Layout& L, uint16_t* out, char* ws,

@@ -225,23 +225,6 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
-// Four rows r0..r3 of a 2-D tensor whose box is one row high (tile::gather4),
-// columns from c0 on, into four consecutive rows of this CTA's shared memory
-// (the tensor map's swizzle applied by address, as for a box); completion is
-// counted on an mbarrier that may live in either CTA of the pair. No multicast.
-__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* map,
-                                                 uint32_t bar_cluster, int32_t c0, int32_t r0,
-                                                 int32_t r1, int32_t r2, int32_t r3,
-                                                 uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      ".cta_group::2.L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(
-          smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
-      "r"(r3), "l"(policy)
-      : "memory");
-}
-
 // 5-D variant (box coordinates c0 innermost .. c4 outermost).
 __device__ __forceinline__ void tma_load_5d_pair(void* dst, const CUtensorMap* map,
                                                  uint32_t bar_cluster, int32_t c0, int32_t c1,

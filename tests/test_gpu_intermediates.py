@@ -9,10 +9,7 @@ and the workspace is read at the offsets beam_moe_workspace_layout reports:
 - pos is the stable grouping by expert: the rows of expert e start at
   offsets[e] and hold its tokens in ascending order (the only permutation the
   library documents), so pos is a bijection onto the A = T K rows;
-- tok (the token of each permuted row) inverts pos, and where the gate/up
-  GEMM reads permuted rows (few rows per expert) they are x[t] byte for byte
-  at pos[t, k]; with many rows per expert the GEMM gathers each row straight
-  from x by tok instead, and h below checks what it read;
+- the permuted rows are x[t] byte for byte at pos[t, k];
 - h at pos[t, k] is the oracle's fp64 silu(Wg x) * (Wu x) after one rounding
   to bf16: within half a bf16 step plus the FP32 accumulation slack stated in
   `_h_slack`, and equal to the correctly rounded value on all but a small
@@ -89,14 +86,6 @@ def _check_dispatch(wl, x, r, ws, lay):
 
 
 def _check_permuted_rows(wl, x, pos, ws, lay):
-    """Every row's token (tok, the inverse of pos) and, when the gate/up GEMM
-    reads permuted rows rather than gathering them from x, every row byte for
-    byte."""
-    tok = _read(ws, lay.tok, np.int32, (wl.T * wl.K,))
-    for k in range(wl.K):
-        assert np.array_equal(tok[pos[:, k]], np.arange(wl.T)), k
-    if lay.gather:
-        return
     xp = _read(ws, lay.xp, np.uint16, (wl.T * wl.K, wl.H))
     for k in range(wl.K):
         assert np.array_equal(xp[pos[:, k]], x), k
@@ -158,7 +147,6 @@ def test_tiny_intermediates(T):
     _check_permuted_rows(wl, x, pos, ws, lay)
     ws, lay = _run_stages(wl, x, 4)
     assert lay.pair_gateup == (1 if T >= 1500 else 0)
-    assert lay.gather == lay.pair_gateup
     _check_h(wl, x, r, ids, pos, ws, lay, np.arange(T))
 
 
