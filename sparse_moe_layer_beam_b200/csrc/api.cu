@@ -81,7 +81,6 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool allow_tc) {
   L.offsets = take(sizeof(int32_t) * (E + 1), 256);
   L.nb_off = take(sizeof(int32_t) * (E + 1), 256);
   L.nb2_off = take(sizeof(int32_t) * (E + 1), 256);
-  L.order = take(sizeof(int32_t) * (2 * (size_t)E + 2), 256);
   L.ids = take(sizeof(int32_t) * (size_t)L.A, 256);
   L.w = take(sizeof(float) * (size_t)L.A, 256);
   L.pos = take(sizeof(int32_t) * (size_t)L.A, 256);
@@ -759,7 +758,7 @@ beam_moe_status ep_checks(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep) {
 // its status word is the workspace's first (shared with the expert stage).
 Layout ep_routing(const beam_moe_cfg& c, int64_t T, int sms, size_t base) {
   Layout L = beam::make_layout(c, T, sms);
-  size_t* f[] = {&L.counts, &L.offsets, &L.nb_off, &L.nb2_off, &L.order, &L.ids, &L.w, &L.pos,
+  size_t* f[] = {&L.counts, &L.offsets, &L.nb_off, &L.nb2_off, &L.ids, &L.w, &L.pos,
                  &L.chunk_cnt, &L.chunk_mask, &L.logits, &L.w3, &L.route_end, &L.xp, &L.h,
                  &L.total};
   for (size_t* v : f) *v += base;

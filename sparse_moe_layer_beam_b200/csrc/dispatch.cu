@@ -63,14 +63,11 @@ __global__ void __launch_bounds__(1024) scan_kernel(const uint32_t* __restrict__
                                                     int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ nb_off,
                                                     int32_t* __restrict__ nb2_off,
-                                                    int32_t* __restrict__ order,
                                                     int32_t* __restrict__ counts_out) {
   __shared__ int32_t part[1024];   // per (team member, expert) partial counts
   __shared__ int32_t s_off[512];   // first row of each expert
-  __shared__ int32_t s_cnt[512];   // rows of each expert
-  __shared__ int32_t s_ord[512];   // experts by class: light ones first
   __shared__ int32_t warp_tot[32];
-  __shared__ int32_t total[5];
+  __shared__ int32_t total[3];
   const int tid = threadIdx.x;
   const int tpe = 1024 / E;  // threads per expert (E <= 512)
   const int e = tid % E, j = tid / E;
@@ -89,26 +86,6 @@ __global__ void __launch_bounds__(1024) scan_kernel(const uint32_t* __restrict__
   const int nbo = block_exclusive_scan(tid < E ? (tot + bn - 1) / bn : 0, warp_tot, &total[1]);
   const int nb2o =
       block_exclusive_scan(tid < E ? (tot + 2 * bn - 1) / (2 * bn) : 0, warp_tot, &total[2]);
-  // experts by class (1..kLightRows rows first, ids ascending in each class)
-  // and the prefix of their token blocks in that order
-  const bool light = tid < E && tot > 0 && tot <= kLightRows;
-  const int lpos = block_exclusive_scan(light ? 1 : 0, warp_tot, &total[3]);
-  const int n_light = total[3];
-  if (tid < E) {
-    s_ord[light ? lpos : n_light + (tid - lpos)] = tid;
-    s_cnt[tid] = tot;
-  }
-  __syncthreads();
-  const int oblk = tid < E ? (s_cnt[s_ord[tid]] + bn - 1) / bn : 0;
-  const int opre = block_exclusive_scan(oblk, warp_tot, &total[4]);
-  if (tid < E) {
-    order[tid] = s_ord[tid];
-    order[E + tid] = opre;
-  }
-  if (tid == 0) {
-    order[2 * E] = total[4];
-    order[2 * E + 1] = n_light;
-  }
   if (tid < E) {
     s_off[tid] = off;
     offsets[tid] = off;
@@ -215,8 +192,7 @@ cudaError_t launch_scan(const beam_moe_cfg& c, const Layout& L, char* ws, int32_
                                   c.n_experts, L.bn, reinterpret_cast<int32_t*>(ws + L.counts),
                                   reinterpret_cast<int32_t*>(ws + L.offsets),
                                   reinterpret_cast<int32_t*>(ws + L.nb_off),
-                                  reinterpret_cast<int32_t*>(ws + L.nb2_off),
-                                  reinterpret_cast<int32_t*>(ws + L.order), counts_out);
+                                  reinterpret_cast<int32_t*>(ws + L.nb2_off), counts_out);
   return cudaGetLastError();
 }
 

@@ -25,7 +25,6 @@
 //  - Every wait is bounded; a timeout sets a status bit and the CTA unwinds
 //    after its own copies and MMAs have completed.
 #include <cuda_bf16.h>
-#include <string.h>
 
 #include "grouped_gemm.cuh"
 #include "internal.h"
@@ -285,7 +284,6 @@ cudaError_t dispatch_bn(int bn, const CUtensorMap& tw, const CUtensorMap& tx, co
 
 GemmParams base_params(const beam_moe_cfg& c, const Layout& L, char* ws) {
   GemmParams p;
-  memset(&p, 0, sizeof(p));
   p.counts = reinterpret_cast<const int32_t*>(ws + L.counts);
   p.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
   p.nb_off = reinterpret_cast<const int32_t*>(ws + L.nb_off);

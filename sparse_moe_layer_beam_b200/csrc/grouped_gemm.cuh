@@ -20,10 +20,6 @@ struct GemmParams {
   int up_rows;  // row offset of the up projection inside an expert (I)
   int n_mblk;   // 128-row weight blocks per expert (I / 128 or H / 128)
   unsigned* status;
-  // Interleaved tile order (CTA-pair GEMMs; null: experts in id order):
-  // order[0..E) experts by class (light first), order[E..2E] the prefix of
-  // token blocks in that order, order[2E + 1] the number of light experts.
-  const int32_t* order;
 };
 
 __host__ __device__ constexpr int pow2_at_least(int v) {

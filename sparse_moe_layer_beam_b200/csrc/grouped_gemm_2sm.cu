@@ -51,59 +51,19 @@ constexpr int kThreads = 192;
 constexpr int kPairM = 256;  // weight rows per pair tile
 constexpr int kPairN = 256;  // max tokens per pair tile (the token block)
 
-// Tile -> (expert, weight block, token block, token blocks of the expert).
-// An expert's tiles run weight block by weight block, so that each weight
-// tile is read from DRAM once while the expert's token rows stay in L2 -
-// unless the token rows outweigh the weights (more rows than the expert has
-// weight rows): then token block by token block, and the weights are what
-// stays in L2.
-//
-// With p.order, the tiles of light experts (1..kLightRows rows, which stream
-// their weights) are spread evenly among the other experts' (compute-bound)
-// tiles: tile t is light when floor((t + 1) NL / N) > floor(t NL / N), NL of
-// N tiles being light, so that at any time some pairs stream weights while
-// the others keep the tensor cores busy. Every role decodes the same way.
+// Tile -> (expert, weight block, token block). An expert's tiles run weight
+// block by weight block, so that each weight tile is read from DRAM once while
+// the expert's token rows stay in L2 - unless the token rows outweigh the
+// weights (more rows than the expert has weight rows): then token block by
+// token block, and the weights are what stays in L2.
 __device__ __forceinline__ void decode_pair_tile(int tile, const GemmParams& p, int& e, int& mb,
-                                                 int& nb, int& nblk) {
-  int lo, hi, base, local;
-  if (p.order) {
-    const int32_t* pre = p.order + p.E;  // token blocks before each position
-    const int n_light = __ldg(p.order + 2 * p.E + 1);
-    const int64_t nl = (int64_t)__ldg(pre + n_light) * p.n_mblk;
-    const int64_t n = (int64_t)__ldg(pre + p.E) * p.n_mblk;
-    const int64_t j = (int64_t)tile * nl / n;
-    const bool is_light = ((int64_t)(tile + 1) * nl / n) > j;
-    const int64_t idx = is_light ? j : nl + (tile - j);  // place in the class order
-    lo = 0;
-    hi = p.E - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if ((int64_t)__ldg(pre + mid) * p.n_mblk <= idx) lo = mid;
-      else hi = mid - 1;
-    }
-    e = __ldg(p.order + lo);
-    base = __ldg(pre + lo);
-    nblk = __ldg(pre + lo + 1) - base;
-    local = (int)(idx - (int64_t)base * p.n_mblk);
-  } else {
-    lo = 0;
-    hi = p.E - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (__ldg(p.nb_off + mid) * p.n_mblk <= tile) lo = mid;
-      else hi = mid - 1;
-    }
-    e = lo;
-    base = __ldg(p.nb_off + e);
-    nblk = __ldg(p.nb_off + e + 1) - base;
-    local = tile - base * p.n_mblk;
-  }
+                                                 int& nb) {
+  decode_tile(tile, p, e, mb, nb);
   if (__ldg(p.counts + e) > p.w_rows) {
+    const int nblk = __ldg(p.nb_off + e + 1) - __ldg(p.nb_off + e);
+    const int local = mb * nblk + nb;
     nb = local / p.n_mblk;
     mb = local - nb * p.n_mblk;
-  } else {
-    mb = local / nblk;
-    nb = local - mb * nblk;
   }
 }
 
@@ -181,14 +141,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t issued = 0;
       bool ok = true;
       for (int tile = pair; tile < total && ok; tile += n_pairs) {
-        int e, mb, nb, nblk;
-        decode_pair_tile(tile, p, e, mb, nb, nblk);
+        int e, mb, nb;
+        decode_pair_tile(tile, p, e, mb, nb);
         const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
         const int half = ((rows + 15) & ~15) >> 1;  // 8 .. 128
         const int xrow = __ldg(p.offsets + e) + nb * kPairN + (int)rank * half;
         const bool box64 = half <= 64;
         const CUtensorMap* tmx = box64 ? &tm_x64 : &tm_x;
         const uint32_t stage_tx = 2u * (uint32_t)(C::kABytes + (box64 ? 64 : 128) * C::kRowBytes);
+        const int nblk = __ldg(p.nb_off + e + 1) - __ldg(p.nb_off + e);
         const uint64_t pol_w = nblk == 1 ? pol_stream : pol_keep;
         // first weight row of this CTA's 128 (down) or first intermediate
         // index of its 64 gate/up pairs
@@ -235,8 +196,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = pair; tile < total && ok; tile += n_pairs) {
-        int e, mb, nb, nblk;
-        decode_pair_tile(tile, p, e, mb, nb, nblk);
+        int e, mb, nb;
+        decode_pair_tile(tile, p, e, mb, nb);
         const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
         const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32(kPairM, n_mma);
@@ -277,8 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < total; tile += n_pairs) {
-      int e, mb, nb, nblk;
-      decode_pair_tile(tile, p, e, mb, nb, nblk);
+      int e, mb, nb;
+      decode_pair_tile(tile, p, e, mb, nb);
       const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
       const int n_mma = (rows + 15) & ~15;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, kFlagEpilogue)) break;
@@ -400,12 +361,8 @@ cudaError_t encode_xmaps(CUtensorMap* m128, CUtensorMap* m64, const void* base, 
   return encode_tmap_2d_bf16(m64, base, cols, rows, kTileK, 64);
 }
 
-// L.order == 0 (a layout built by hand, as expert parallelism does): tiles in
-// expert id order.
 GemmParams base_params(const beam_moe_cfg& c, const Layout& L, char* ws) {
   GemmParams p;
-  memset(&p, 0, sizeof(p));
-  p.order = L.order ? reinterpret_cast<const int32_t*>(ws + L.order) : nullptr;
   p.counts = reinterpret_cast<const int32_t*>(ws + L.counts);
   p.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
   p.nb_off = reinterpret_cast<const int32_t*>(ws + L.nb_off);

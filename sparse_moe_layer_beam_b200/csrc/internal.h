@@ -17,12 +17,6 @@ namespace beam {
 constexpr int kChunk = 128;
 constexpr int kChunkWords = kChunk / 32;
 
-// Experts with at most this many rows make memory-bound tiles on the GEMMs
-// (each weight byte feeds fewer FLOPs than the tensor cores can do while
-// HBM delivers it); the CTA-pair GEMMs spread their tiles evenly among the
-// others' so that weight streaming overlaps the compute-bound tiles.
-constexpr int kLightRows = 128;
-
 // Rows of weights per tensor-core tile (the MMA M dimension) and the K step
 // of one pipeline stage (64 bf16 = one 128-byte swizzle row).
 constexpr int kTileM = 128;
@@ -89,9 +83,6 @@ struct Layout {
   size_t offsets;   // int32[E + 1] first row of each expert in the permuted rows
   size_t nb_off;    // int32[E + 1] prefix of ceil(count / bn)
   size_t nb2_off;   // int32[E + 1] prefix of ceil(count / (2 bn))
-  size_t order;     // int32[2 E + 2] experts with 1..kLightRows rows, then the
-                    // others (ids ascending in each class); the prefix of
-                    // ceil(count / bn) in that order [E + 1]; the light count
   size_t ids;       // int32[T * K]
   size_t w;         // float[T * K]
   size_t pos;       // int32[T * K] permuted row of each assignment
