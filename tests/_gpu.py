@@ -295,6 +295,22 @@ def check_nvfp4(out_bits, ref):
     assert rms_excess <= TOL_NVFP4_RMS, (rms_excess, rms)
 
 
+def combine_bits(y, pos, w):
+    """bf16 bits of out[t] = sum_k w[t, k] y[pos[t, k]]: a chain of FP32 fused
+    multiply-adds in ascending k (pos < 0 skipped) from 0, rounded once to
+    bf16 (nearest, ties to even). Each step forms the exact product plus the
+    running sum in extended precision and rounds it to FP32 once."""
+    T, K = pos.shape
+    acc = np.zeros((T, y.shape[1]), np.float32)
+    for k in range(K):
+        p = pos[:, k]
+        ok = p >= 0
+        prod = w[ok, k].astype(np.longdouble)[:, None] * y[p[ok]].astype(np.longdouble)
+        acc[ok] = (prod + acc[ok].astype(np.longdouble)).astype(np.float32)
+    u = acc.view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
 def max_rel_err(out_bits, ref):
     got = synth.bf16_to_f32(out_bits).astype(np.float64)
     rms = np.sqrt(np.mean(ref ** 2))

@@ -14,7 +14,9 @@ and the workspace is read at the offsets beam_moe_workspace_layout reports:
   to bf16: within half a bf16 step plus the FP32 accumulation slack stated in
   `_h_slack`, and equal to the correctly rounded value on all but a small
   fraction of elements (those whose exact value lies within that slack of a
-  rounding midpoint).
+  rounding midpoint);
+- out is the k-ordered FP32 sum of the y rows the workspace holds, bit for
+  bit, after either down GEMM (one CTA per tile or CTA pairs).
 """
 import numpy as np
 import pytest
@@ -187,3 +189,24 @@ def test_all_stages_equal_the_forward():
     bm.beam_moe_forward_stages(cfg, _gpu.to_dev_bits(x), wr, None, w13, w2, out, 6, ws)
     assert bm.beam_moe_check(ws) == 0
     assert np.array_equal(_gpu.bits_of(out), g["out"])
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 200), ("tiny", 1500), ("prefill", None)])
+def test_combine_is_the_k_ordered_fp32_sum(name, T):
+    """T = 200: y from the one-CTA down GEMM; 1500 and prefill (Beam's shape):
+    y from the down GEMM on CTA pairs."""
+    wl = synth.workload(name) if T is None else synth.workload(name).with_T(T)
+    x = synth.host_x(wl)
+    cfg = _gpu.cfg_of(wl)
+    w13, w2, wr = _gpu.device_weights(wl)
+    out = torch.empty((wl.T, wl.H), dtype=torch.int16, device="cuda")
+    ws = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T), dtype=torch.uint8, device="cuda")
+    bm.beam_moe_forward_stages(cfg, _gpu.to_dev_bits(x), wr, None, w13, w2, out, 6, ws)
+    assert bm.beam_moe_check(ws) == 0
+    lay = bm.beam_moe_workspace_layout(cfg, wl.T)
+    assert lay.pair_down == (0 if wl.T == 200 else 1)
+    A = wl.T * wl.K
+    pos = _read(ws, lay.pos, np.int32, (wl.T, wl.K))
+    w = _read(ws, lay.w, np.float32, (wl.T, wl.K))
+    y = _read(ws, lay.y, np.float32, (A, wl.H))
+    assert np.array_equal(_gpu.bits_of(out), _gpu.combine_bits(y, pos, w))

@@ -170,6 +170,36 @@ def test_routed_forward_matches_oracle():
     assert bm.beam_moe_check(ws) & 0x100
 
 
+def test_routed_forward_on_cta_pairs_with_dropped_and_repeated_ids():
+    """Routing replay with both grouped GEMMs on CTA pairs: an out-of-range id
+    drops its assignment (flag 0x100), a token with no valid id gets a zero
+    row, and a repeated id (outside the call's contract of distinct ids) adds
+    the expert's output once per slot, as the oracle's sum does."""
+    wl = synth.workload("tiny").with_T(600)
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    cfg = _gpu.cfg_of(wl)
+    assert bm.beam_moe_workspace_layout(cfg, wl.T).pair_down == 1
+    w13, w2, _ = _gpu.device_weights(wl)
+    ids = r["ids"].astype(np.int32).copy()
+    w = r["weights"].astype(np.float32).copy()
+    ids[3, 1] = wl.E + 5
+    ids[5, :] = -1
+    ids[7, 2] = ids[7, 0]
+    ids[9, :] = ids[9, 0]
+    out = torch.empty((wl.T, wl.H), dtype=torch.int16, device="cuda")
+    ws = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T), dtype=torch.uint8, device="cuda")
+    bm.beam_moe_forward_routed(cfg, _gpu.to_dev_bits(x), torch.from_numpy(ids).cuda(),
+                               torch.from_numpy(w).cuda(), w13, w2, out, ws, None)
+    assert bm.beam_moe_check(ws) & 0x100
+    got = _gpu.bits_of(out)
+    assert not got[5].any()  # no valid id: a zero row
+    bad = (ids < 0) | (ids >= wl.E)
+    ref = oracle.experts(oracle.cfg_for(wl), x, np.where(bad, 0, ids), np.where(bad, 0.0, w),
+                         synth.host_w13(wl), synth.host_w2(wl))
+    err, _ = _gpu.max_rel_err(got, ref)
+    assert err <= _gpu.TOL
+
+
 def test_route_only_entry_point():
     wl = synth.workload("decode").with_T(300)
     x, _, wr, b, r = _inputs.routed_inputs(wl)
