@@ -522,7 +522,9 @@ def run_ep(args, wl):
     tokens, exchanges workspaces once through CUDA IPC, and per step
     all-gathers the counts (NCCL), plans on the host, dispatches by peer
     stores, runs its experts (y rows stored back into their sources) and
-    combines, with a barrier after the dispatch and after the experts."""
+    combines. No barrier between dispatch and experts: the gate/up GEMM waits
+    for each expert's rows on the arrival counters the dispatch increments;
+    one barrier after the experts."""
     import datetime
 
     import torch
@@ -581,7 +583,6 @@ def run_ep(args, wl):
         send_base, recv_counts, _ = bm.beam_moe_ep_plan(cfg, ep, counts_all)
         bm.beam_moe_ep_dispatch(cfg, ep, x, torch.from_numpy(send_base).to(dev, non_blocking=True),
                                 peers.ptrs, ws, stream=st)
-        barrier()
         bm.beam_moe_ep_experts(cfg, ep, recv_counts, w13, w2, peers.ptrs, ws, stream=st)
         barrier()
         bm.beam_moe_ep_combine(cfg, ep, wl.T, out, ws, stream=st)

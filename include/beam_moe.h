@@ -337,16 +337,27 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_traced(const beam_moe_cfg* cfg, in
  *   2 beam_moe_ep_plan      (host) where this rank's rows land in every
  *                           owner's receive buffer, and what it receives
  *   3 beam_moe_ep_dispatch  writes its token rows and their return
- *                           addresses into the owners' workspaces
- *   -                       barrier: every rank's dispatch has completed
+ *                           addresses into the owners' workspaces and
+ *                           counts each row on its owner's arrival counter
+ *                           of the row's expert (system-scope atomics)
  *   4 beam_moe_ep_experts   grouped GEMMs over the received rows, each y row
  *                           written back into its source rank's workspace
  *                           (from the down GEMM's epilogue when it runs on
- *                           CTA pairs, else by a copy kernel after it)
+ *                           CTA pairs, else by a copy kernel after it). No
+ *                           barrier is needed before it: the gate/up GEMM
+ *                           starts on an expert's rows once its arrival
+ *                           counter reaches recv_counts, so it overlaps the
+ *                           other ranks' dispatch
  *   -                       barrier: every rank's experts call has completed
  *   5 beam_moe_ep_combine   out[t] = sum_k w[t][k] y[t][k], fixed k order
- * No kernel waits for another rank: the caller orders the phases (an NCCL
- * all-gather and barriers, or stream order when all ranks share one GPU).
+ * The arrival wait is the one place a kernel waits for another rank. It is
+ * bounded: after 1 s without the rows it sets status bit 0x1000 and goes on
+ * with whatever the buffer holds. Ranks must therefore run on different GPUs
+ * (or, when several share one GPU, be ordered by the caller so that every
+ * dispatch has completed before any experts call starts: kernels of
+ * different processes on one GPU need not run at the same time). The route
+ * call clears the rank's arrival counters; no rank may dispatch to it before
+ * the counts of that route call have been gathered.
  * peer_ws[r] is rank r's workspace as a pointer this rank's GPU can store
  * to (NVLink peer memory; the same allocation when r == rank). Every rank's
  * workspace has the same size and layout (same cfg, world, t_max,
@@ -448,7 +459,9 @@ BEAM_MOE_API beam_moe_status beam_moe_ep_release(const beam_moe_ep_handle* handl
  * is not stored; only inconsistent recv_counts lead there); 0x800 a
  * dispatched row's place in its owner's receive buffer fell outside
  * [0, recv_cap) (the row is not stored; send_base from another step's plan
- * leads there). Returns
+ * leads there); 0x1000 an expert's received rows did not all arrive within
+ * 1 s of the experts call's gate/up GEMM asking for them (recv_counts larger
+ * than what the ranks dispatched, or a rank that never dispatched). Returns
  * BEAM_MOE_ERR_DEVICE_TIMEOUT
  * if any bit was set, BEAM_MOE_ERR_CUDA if the stream reports an error.
  */

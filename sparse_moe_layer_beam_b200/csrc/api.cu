@@ -839,13 +839,16 @@ beam_moe_status beam_moe_ep_route(const beam_moe_cfg* cfg, const beam_moe_ep_cfg
   BEAM_TRY(check_ptrs({counts}, {}));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
+  const beam::EpLayout P = beam::make_ep_layout(*cfg, *ep);
   BEAM_CUDA(cudaMemsetAsync(w, 0, 256, st));
+  // arrival counters of this step: no rank dispatches here before the counts
+  // of this call have been gathered
+  BEAM_CUDA(cudaMemsetAsync(w + P.arrive, 0, 4 * (size_t)(cfg->n_experts / ep->world), st));
   if (T == 0) {
     BEAM_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, st));
     return BEAM_MOE_OK;
   }
   BEAM_TRY(check_ptrs({x, w_router}, {bias}));
-  const beam::EpLayout P = beam::make_ep_layout(*cfg, *ep);
   const Layout L = ep_routing(*cfg, T, beam::device_sm_count(), P.route);
   BEAM_CUDA(beam::launch_router_logits(*cfg, L, x, w_router, w, st));
   BEAM_CUDA(beam::launch_router_topk(*cfg, L, bias, w, st));
@@ -950,6 +953,7 @@ beam_moe_status beam_moe_ep_experts(const beam_moe_cfg* cfg, const beam_moe_ep_c
   L.nb_off = P.nb_off;
   L.xp = P.recv;
   L.h = P.h;
+  L.arrive = P.arrive;  // gate/up waits for each expert's rows from the other ranks
   int32_t acc = 0;
   for (int j = 0; j < El; ++j) {
     nb_off[j] = acc;

@@ -8,18 +8,24 @@
 //             rows land in each owner's receive buffer;
 //   dispatch  each rank writes its token rows straight into the owners'
 //             receive buffers with peer stores (NVLink), plus the row's return
-//             address (source rank, token slot);
-//   experts   each rank runs the grouped GEMMs over the rows it received and
-//             writes every y row back into its source rank's buffer;
+//             address (source rank, token slot), and counts every row on its
+//             owner's per-expert arrival counter;
+//   experts   each rank runs the grouped GEMMs over the rows it received,
+//             starting on an expert's rows as soon as its counter shows them
+//             all (no barrier between dispatch and experts), and writes every
+//             y row back into its source rank's buffer;
 //   combine   each rank sums its tokens' K returned rows with the weights.
 //
-// The caller orders the phases across ranks (an all-gather of the counts
-// between route and plan, a barrier after dispatch and after experts); no
-// kernel waits for another rank. Every rank's workspace has the same layout,
+// The caller orders the other phases across ranks (an all-gather of the
+// counts between route and plan, a barrier after experts). The gate/up GEMM's
+// wait for arrivals is the only place a kernel waits for another rank; it is
+// bounded (1 s, then status bit kFlagArrival). Every rank's workspace has the
+// same layout,
 // so a peer's buffer is its workspace pointer plus a fixed offset: [status]
 // [receive rows: cap x H x 4 bytes, bf16 on arrival, fp32 y after the down
 // GEMM][return addresses: cap x int32][returned y: T_max K x H fp32][h: cap x
-// I bf16][local expert counts, offsets, token-tile prefix][routing scratch].
+// I bf16][local expert counts, offsets, token-tile prefix][arrival counters: E / world
+// int32][routing scratch].
 #include <string.h>
 
 #include "internal.h"
@@ -57,6 +63,7 @@ EpLayout make_ep_layout(const beam_moe_cfg& c, const beam_moe_ep_cfg& g) {
   P.counts = take(4 * (size_t)El, 256);
   P.offsets = take(4 * (size_t)(El + 1), 256);
   P.nb_off = take(4 * (size_t)(El + 1), 256);
+  P.arrive = take(4 * (size_t)El, 256);
   P.route = up(o, 1024);
   return P;
 }
@@ -64,7 +71,9 @@ EpLayout make_ep_layout(const beam_moe_cfg& c, const beam_moe_ep_cfg& g) {
 namespace {
 
 // One CTA per local token: the K return addresses and combine positions,
-// then the token's row copied to each owner's receive buffer. A row whose
+// then the token's row copied to each owner's receive buffer and counted on
+// the owner's arrival counter of its expert (after a system-scope fence, so
+// an owner that sees the count sees the row). A row whose
 // place in the owner's buffer falls outside [0, recv_cap) (send_base from
 // another step's plan, for instance) is never stored: it is dropped, its
 // combine position is -1 and status bit kFlagBadDispatch is set.
@@ -74,14 +83,16 @@ __global__ void __launch_bounds__(128) ep_dispatch_kernel(
     const uint32_t* __restrict__ chunk_mask, const int32_t* __restrict__ offsets,
     const int32_t* __restrict__ send_base, int32_t* __restrict__ pos,
     const __grid_constant__ Peers peers,
-    size_t recv_off, size_t src_off, int64_t recv_cap, unsigned* status) {
+    size_t recv_off, size_t src_off, size_t arrive_off, int64_t recv_cap, unsigned* status) {
   __shared__ uint16_t* s_dst[32];
+  __shared__ int32_t* s_arrive[32];
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
   if (tid < K) {
     const size_t slot = (size_t)t * K + tid;
     const int e = ids[slot];
     uint16_t* dst = nullptr;
+    int32_t* arr = nullptr;
     if (e >= 0 && e < E) {
       const int c = t / kChunk, tl = t - c * kChunk;
       const uint32_t* m = chunk_mask + ((size_t)c * E + e) * kChunkWords;
@@ -93,6 +104,7 @@ __global__ void __launch_bounds__(128) ep_dispatch_kernel(
       if (row >= 0 && row < recv_cap) {
         char* peer = peers.ws[e / El];
         dst = reinterpret_cast<uint16_t*>(peer + recv_off) + (size_t)row * H;
+        arr = reinterpret_cast<int32_t*>(peer + arrive_off) + (e % El);
         reinterpret_cast<int32_t*>(peer + src_off)[row] = (rank << kSlotBits) | (int)slot;
         pos[slot] = (int)slot;
       } else {
@@ -103,6 +115,7 @@ __global__ void __launch_bounds__(128) ep_dispatch_kernel(
       pos[slot] = -1;
     }
     s_dst[tid] = dst;
+    s_arrive[tid] = arr;
   }
   __syncthreads();
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
@@ -111,8 +124,10 @@ __global__ void __launch_bounds__(128) ep_dispatch_kernel(
     if (!d) continue;
     for (int v = tid; v < H / 8; v += 128) d[v] = __ldg(src + v);
   }
-  // the owners read these rows in their next phase, on other GPUs
+  // every store of this CTA reaches the owners (other GPUs) before its count
   __threadfence_system();
+  __syncthreads();
+  if (tid < K && s_arrive[tid]) atomicAdd_system(s_arrive[tid], 1);
 }
 
 // Every received y row back to its source rank's returned-y buffer.
@@ -153,7 +168,7 @@ cudaError_t launch_ep_dispatch(const beam_moe_cfg& c, const beam_moe_ep_cfg& g,
       reinterpret_cast<const int32_t*>(wr + L.ids), reinterpret_cast<const int32_t*>(wr + L.chunk_cnt),
       reinterpret_cast<const uint32_t*>(wr + L.chunk_mask),
       reinterpret_cast<const int32_t*>(wr + L.offsets), send_base,
-      reinterpret_cast<int32_t*>(wr + L.pos), peers, P.recv, P.src, g.recv_cap,
+      reinterpret_cast<int32_t*>(wr + L.pos), peers, P.recv, P.src, P.arrive, g.recv_cap,
       reinterpret_cast<unsigned*>(wr + P.status));
   return cudaGetLastError();
 }

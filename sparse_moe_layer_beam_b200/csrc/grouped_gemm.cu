@@ -100,6 +100,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // A producer may spend up to its 1 s arrival limit waiting for rows from
+  // other ranks; the other roles' waits allow for that.
+  const uint64_t wait_ns = p.arrive ? 3000000000ull : 1000000000ull;
   const int total = __ldg(p.nb_off + p.E) * p.n_mblk;
 
   if (warp == 0) {
@@ -114,15 +117,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int64_t issued = 0;
       bool ok = true;
+      int arrived_e = -1;  // the expert whose rows are known to be here
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int e, mb, nb;
         decode_tile(tile, p, e, mb, nb);
+        if (p.arrive && e != arrived_e) {
+          rows_arrived(p.arrive + e, __ldg(p.counts + e), p.status, kFlagArrival);
+          arrived_e = e;
+        }
         const int wrow = e * p.w_rows + mb * kTileM;
         const int xrow = __ldg(p.offsets + e) + nb * BN;
         const int nblk = __ldg(p.nb_off + e + 1) - __ldg(p.nb_off + e);
         const uint64_t pol_w = nblk == 1 ? pol_stream : pol_keep;
         for (int kb = 0; kb < p.nk; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, kFlagProducer)) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, kFlagProducer, wait_ns)) {
             ok = false;
             break;
           }
@@ -161,12 +169,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rows = min(BN, __ldg(p.counts + e) - nb * BN);
         const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32(kTileM, n_mma);
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, kFlagMma)) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, kFlagMma, wait_ns)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + (uint32_t)(acc * C::kAccCols);
         const uint32_t d1 = d0 + BN;
         for (int kb = 0; kb < p.nk; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, kFlagMma)) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, kFlagMma, wait_ns)) {
             ok = false;
             break;
           }
@@ -212,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       decode_tile(tile, p, e, mb, nb);
       const int rows = min(BN, __ldg(p.counts + e) - nb * BN);
       const int n_mma = (rows + 15) & ~15;
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, kFlagEpilogue)) break;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, kFlagEpilogue, wait_ns)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
       const int64_t row0 = __ldg(p.offsets + e) + nb * BN;
@@ -289,6 +297,7 @@ GemmParams base_params(const beam_moe_cfg& c, const Layout& L, char* ws) {
   p.nb_off = reinterpret_cast<const int32_t*>(ws + L.nb_off);
   p.E = c.n_experts;
   p.status = reinterpret_cast<unsigned*>(ws + L.status);
+  p.arrive = L.arrive ? reinterpret_cast<const int32_t*>(ws + L.arrive) : nullptr;
   return p;
 }
 
@@ -326,6 +335,7 @@ cudaError_t launch_down(const beam_moe_cfg& c, const Layout& L, const uint16_t* 
   p.nk = I / kTileK;
   p.w_rows = H;
   p.up_rows = 0;
+  p.arrive = nullptr;  // h rows are this rank's own
   p.n_mblk = H / kTileM;
   return dispatch_bn<false>(L.bn, tw, tx, p, st);
 }

@@ -20,6 +20,8 @@ struct GemmParams {
   int up_rows;  // row offset of the up projection inside an expert (I)
   int n_mblk;   // 128-row weight blocks per expert (I / 128 or H / 128)
   unsigned* status;
+  const int32_t* arrive;  // [E] or nullptr: rows arrived per expert (expert parallelism);
+                          // a tile's rows are loaded once arrive[e] reaches counts[e]
 };
 
 __host__ __device__ constexpr int pow2_at_least(int v) {

@@ -129,6 +129,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // A producer may spend up to its 1 s arrival limit waiting for rows from
+  // other ranks; the other roles' waits allow for that.
+  const uint64_t wait_ns = p.arrive ? 3000000000ull : 1000000000ull;
   const int total = __ldg(p.nb_off + p.E) * p.n_mblk;
 
   if (warp == 0) {
@@ -140,9 +143,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int64_t issued = 0;
       bool ok = true;
+      int arrived_e = -1;  // the expert whose rows are known to be here
       for (int tile = pair; tile < total && ok; tile += n_pairs) {
         int e, mb, nb;
         decode_pair_tile(tile, p, e, mb, nb);
+        if (p.arrive && e != arrived_e) {
+          rows_arrived(p.arrive + e, __ldg(p.counts + e), p.status, kFlagArrival);
+          arrived_e = e;
+        }
         const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
         const int half = ((rows + 15) & ~15) >> 1;  // 8 .. 128
         const int xrow = __ldg(p.offsets + e) + nb * kPairN + (int)rank * half;
@@ -156,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int w0 = GATEUP ? mb * 128 + (int)rank * 64
                               : e * p.w_rows + mb * kPairM + (int)rank * 128;
         for (int kb = 0; kb < p.nk; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, kFlagProducer)) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, kFlagProducer, wait_ns)) {
             ok = false;
             break;
           }
@@ -201,11 +209,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
         const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32(kPairM, n_mma);
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, kFlagMma)) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, kFlagMma, wait_ns)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(acc * C::kAccCols);
         for (int kb = 0; kb < p.nk; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, kFlagMma)) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, kFlagMma, wait_ns)) {
             ok = false;
             break;
           }
@@ -242,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       decode_pair_tile(tile, p, e, mb, nb);
       const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
       const int n_mma = (rows + 15) & ~15;
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, kFlagEpilogue)) break;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, kFlagEpilogue, wait_ns)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::kAccCols);
       const int64_t row0 = __ldg(p.offsets + e) + nb * kPairN;
@@ -368,6 +376,7 @@ GemmParams base_params(const beam_moe_cfg& c, const Layout& L, char* ws) {
   p.nb_off = reinterpret_cast<const int32_t*>(ws + L.nb_off);
   p.E = c.n_experts;
   p.status = reinterpret_cast<unsigned*>(ws + L.status);
+  p.arrive = L.arrive ? reinterpret_cast<const int32_t*>(ws + L.arrive) : nullptr;
   return p;
 }
 
@@ -411,6 +420,7 @@ cudaError_t launch_down_pair(const beam_moe_cfg& c, const Layout& L, const uint1
   p.nk = I / kTileK;
   p.w_rows = H;
   p.up_rows = 0;
+  p.arrive = nullptr;  // h rows are this rank's own
   p.n_mblk = H / kPairM;
   if (ret && ret->src) return run_pair<false, true>(tw, tx, tx64, p, *ret, st);
   EpReturn none;

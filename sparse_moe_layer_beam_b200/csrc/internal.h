@@ -30,6 +30,7 @@ constexpr uint32_t kFlagBadExpert = 0x100;
 constexpr uint32_t kFlagSelftest = 0x200;  // beam_moe_selftest_wait's wait ran out
 constexpr uint32_t kFlagBadReturn = 0x400; // a received row's return address out of range
 constexpr uint32_t kFlagBadDispatch = 0x800; // a dispatched row would land outside recv_cap
+constexpr uint32_t kFlagArrival = 0x1000;    // an expert's received rows did not all arrive
 
 // A value set up once per device (a kernel's shared-memory attribute, the
 // number of CTA pairs that can be resident), for host code that launches on
@@ -93,6 +94,7 @@ struct Layout {
   size_t route_end; // bytes needed by the routing op
   size_t xp;        // bf16[A * H] permuted rows; reused for the down output y, fp32[A * H]
   size_t h;         // bf16[A * I] SwiGLU activations
+  size_t arrive;    // int32[E] rows of each expert arrived from other ranks (0: none to wait for)
   size_t total;     // bytes needed by the forward op
 };
 
@@ -136,7 +138,7 @@ struct EpReturn {
 };
 
 struct EpLayout {
-  size_t status, recv, src, yret, h, counts, offsets, nb_off, route;
+  size_t status, recv, src, yret, h, counts, offsets, nb_off, arrive, route;
 };
 EpLayout make_ep_layout(const beam_moe_cfg& c, const beam_moe_ep_cfg& g);
 

@@ -73,6 +73,41 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Expert parallelism: wait until *arrive (rows other ranks have stored here
+// and counted with system-scope atomics) reaches want, then order those rows
+// before this thread's TMA reads of them. Gives up after limit_ns, or as soon
+// as another CTA has (its bit in *status): sets `flag` and returns false; the
+// caller goes on, and the status word reports the failure.
+__device__ __forceinline__ int ld_acquire_sys(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.sys.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ bool rows_arrived(const int32_t* arrive, int want, unsigned* status,
+                                             uint32_t flag, uint64_t limit_ns = 1000000000ull) {
+  bool ok = ld_acquire_sys(arrive) >= want;
+  if (!ok) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+      if (ld_acquire_sys(arrive) >= want) {
+        ok = true;
+        break;
+      }
+      if ((i & 63u) == 0) {
+        if (*reinterpret_cast<volatile unsigned*>(status) & flag) break;
+        if (global_timer_ns() - t0 > limit_ns) {
+          atomicOr(status, flag);
+          break;
+        }
+      }
+      __nanosleep(100);
+    }
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return ok;
+}
+
 // ------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -2,9 +2,11 @@
 one GPU and reach each other's workspaces through the library's CUDA IPC
 calls (beam_moe_ep_export / import / release, exchanged with an all-gather
 over a gloo process group), exactly as ranks on different GPUs do over NVLink.
-No kernel waits for another rank: the phases are ordered on the host (device
-synchronisation, then a gloo barrier), so the two processes never depend on
-each other's kernels running at the same time. Each rank's output must match
+The phases are ordered on the host (device synchronisation, then a gloo
+barrier, also after the dispatch): two processes sharing one GPU must not
+depend on each other's kernels running at the same time, so every row has
+arrived before either experts call starts and its arrival wait returns at
+once. Each rank's output must match
 the oracle and a single-process forward of the same tokens.
 
 "Welcome Beam" (section "Mixture of Experts") and the vLLM recipe page run
