@@ -489,8 +489,10 @@ def measure(args, wl, ex, dev, stream, rank, world, local):
     roof["traffic"] = None if nvfp4 else gateup_traffic(wl, alg)
     # router GEMM (plus the weight split on tensor cores), top-k, scan,
     # permute, gate/up, down, combine; replayed routes: the route copy, scan,
-    # permute, gate/up, down, combine
-    per_step = 6 if args.replay else (8 if lay.router_tc else 7)
+    # permute, gate/up, down, combine; the light experts' one-CTA gate/up and
+    # down after the CTA-pair ones
+    per_step = ((6 if args.replay else (8 if lay.router_tc else 7))
+                + (2 if lay.light_rows and not nvfp4 else 0))
     part = {
         "value": value, "ms_per_step": ms_step,
         "config": {"workload": describe(wl) + (" [routes replayed]" if args.replay else "")

@@ -290,6 +290,9 @@ typedef struct beam_moe_ws_layout {
   int32_t router_tc;     /* 1: the router GEMM runs on tensor cores           */
   int32_t pair_gateup;   /* 1: gate/up grouped GEMM on CTA pairs              */
   int32_t pair_down;     /* 1: down grouped GEMM on CTA pairs                 */
+  int32_t light_rows;    /* with CTA pairs: experts with at most this many
+                            rows run on one-CTA tiles, after the CTA-pair
+                            GEMMs (they only stream weights); 0: none       */
 } beam_moe_ws_layout;
 BEAM_MOE_API beam_moe_status beam_moe_workspace_layout(const beam_moe_cfg* cfg, int64_t T,
                                                        beam_moe_op op,
@@ -304,7 +307,9 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_stages(
  * it is passed to: slot i of stage s is the time of that stage in the i-th
  * traced call since the last reset. Stages: 0 router GEMM, 1 top-k and
  * chunk counts, 2 scan, 3 permute, 4 gate/up grouped GEMM, 5 down grouped
- * GEMM, 6 combine. beam_moe_trace_read synchronizes the recorded events.
+ * GEMM, 6 combine (a GEMM stage holds both of its launches when light
+ * experts run on one-CTA tiles). beam_moe_trace_read synchronizes the
+ * recorded events.
  */
 #define BEAM_MOE_N_STAGES 7
 typedef struct beam_moe_trace beam_moe_trace;

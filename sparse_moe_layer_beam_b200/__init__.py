@@ -56,7 +56,7 @@ class BeamMoeWsLayout(ctypes.Structure):
                 ("w", ctypes.c_int64), ("pos", ctypes.c_int64), ("xp", ctypes.c_int64),
                 ("h", ctypes.c_int64), ("y", ctypes.c_int64), ("router_splits", ctypes.c_int32),
                 ("router_tc", ctypes.c_int32), ("pair_gateup", ctypes.c_int32),
-                ("pair_down", ctypes.c_int32)]
+                ("pair_down", ctypes.c_int32), ("light_rows", ctypes.c_int32)]
 
 
 class BeamMoeNvfp4Experts(ctypes.Structure):

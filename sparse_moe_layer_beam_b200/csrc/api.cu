@@ -68,6 +68,12 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool allow_tc) {
   const bool pair_ok = L.bn == 256 && pair_gemm_supported(c);
   L.pair_gateup = (pair_ok && mean_rows >= 64.0) ? 1 : 0;
   L.pair_down = (pair_ok && mean_rows >= 64.0) ? 1 : 0;
+  // Experts with few rows only stream their weights; a pair tile of 256
+  // weight rows does that at about 0.7 of HBM, the one-CTA kernel (128
+  // weight rows, one 64-token tile) close to 1. With pairs on, such experts
+  // run there, after the others.
+  L.light_max = L.pair_gateup ? kLightRows : 0;
+  L.light_bn = kLightRows;
 
   size_t o = 0;
   auto take = [&](size_t bytes, size_t align) {
@@ -81,6 +87,7 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool allow_tc) {
   L.offsets = take(sizeof(int32_t) * (E + 1), 256);
   L.nb_off = take(sizeof(int32_t) * (E + 1), 256);
   L.nb2_off = take(sizeof(int32_t) * (E + 1), 256);
+  L.nbl_off = take(sizeof(int32_t) * (E + 1), 256);
   L.ids = take(sizeof(int32_t) * (size_t)L.A, 256);
   L.w = take(sizeof(float) * (size_t)L.A, 256);
   L.pos = take(sizeof(int32_t) * (size_t)L.A, 256);
@@ -291,10 +298,12 @@ beam_moe_status expert_path(const beam_moe_cfg* cfg, const Layout& L, const uint
   if (last < 4) return BEAM_MOE_OK;
   BEAM_CUDA(L.pair_gateup ? beam::launch_gateup_pair(*cfg, L, w13, ws, st)
                           : beam::launch_gateup(*cfg, L, w13, ws, st));
+  if (L.light_max) BEAM_CUDA(beam::launch_gateup_light(*cfg, L, w13, ws, st));
   BEAM_CUDA(rec.mark(5));
   if (last < 5) return BEAM_MOE_OK;
   BEAM_CUDA(L.pair_down ? beam::launch_down_pair(*cfg, L, w2, ws, st)
                         : beam::launch_down(*cfg, L, w2, ws, st));
+  if (L.light_max) BEAM_CUDA(beam::launch_down_light(*cfg, L, w2, ws, st));
   BEAM_CUDA(rec.mark(6));
   if (last < 6) return BEAM_MOE_OK;
   BEAM_CUDA(beam::launch_combine(*cfg, L, out, ws, st));
@@ -656,6 +665,7 @@ beam_moe_status beam_moe_workspace_layout(const beam_moe_cfg* cfg, int64_t T, be
   out->router_tc = L.router_tc;
   out->pair_gateup = L.pair_gateup;
   out->pair_down = L.pair_down;
+  out->light_rows = L.light_max;
   return BEAM_MOE_OK;
 }
 
@@ -758,7 +768,7 @@ beam_moe_status ep_checks(const beam_moe_cfg* cfg, const beam_moe_ep_cfg* ep) {
 // its status word is the workspace's first (shared with the expert stage).
 Layout ep_routing(const beam_moe_cfg& c, int64_t T, int sms, size_t base) {
   Layout L = beam::make_layout(c, T, sms);
-  size_t* f[] = {&L.counts, &L.offsets, &L.nb_off, &L.nb2_off, &L.ids, &L.w, &L.pos,
+  size_t* f[] = {&L.counts, &L.offsets, &L.nb_off, &L.nb2_off, &L.nbl_off, &L.ids, &L.w, &L.pos,
                  &L.chunk_cnt, &L.chunk_mask, &L.logits, &L.w3, &L.route_end, &L.xp, &L.h,
                  &L.total};
   for (size_t* v : f) *v += base;

@@ -57,17 +57,21 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
   return r;
 }
 
+// light_max > 0: experts with at most light_max rows get no bn-blocks in
+// nb_off and ceil(count / lbn) blocks in nbl_off (the others none there).
 __global__ void __launch_bounds__(1024) scan_kernel(const uint32_t* __restrict__ bits,
                                                     int32_t* __restrict__ chunk_base, int nchunks,
                                                     int E, int bn, int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ nb_off,
                                                     int32_t* __restrict__ nb2_off,
+                                                    int light_max, int lbn,
+                                                    int32_t* __restrict__ nbl_off,
                                                     int32_t* __restrict__ counts_out) {
   __shared__ int32_t part[1024];   // per (team member, expert) partial counts
   __shared__ int32_t s_off[512];   // first row of each expert
   __shared__ int32_t warp_tot[32];
-  __shared__ int32_t total[3];
+  __shared__ int32_t total[4];
   const int tid = threadIdx.x;
   const int tpe = 1024 / E;  // threads per expert (E <= 512)
   const int e = tid % E, j = tid / E;
@@ -82,15 +86,19 @@ __global__ void __launch_bounds__(1024) scan_kernel(const uint32_t* __restrict__
   int tot = 0;
   if (tid < E)
     for (int q = 0; q < tpe; ++q) tot += part[q * E + tid];
+  const bool light = tid < E && light_max > 0 && tot <= light_max;
   const int off = block_exclusive_scan(tid < E ? tot : 0, warp_tot, &total[0]);
-  const int nbo = block_exclusive_scan(tid < E ? (tot + bn - 1) / bn : 0, warp_tot, &total[1]);
+  const int nbo =
+      block_exclusive_scan(tid < E && !light ? (tot + bn - 1) / bn : 0, warp_tot, &total[1]);
   const int nb2o =
       block_exclusive_scan(tid < E ? (tot + 2 * bn - 1) / (2 * bn) : 0, warp_tot, &total[2]);
+  const int nblo = block_exclusive_scan(light ? (tot + lbn - 1) / lbn : 0, warp_tot, &total[3]);
   if (tid < E) {
     s_off[tid] = off;
     offsets[tid] = off;
     nb_off[tid] = nbo;
     nb2_off[tid] = nb2o;
+    nbl_off[tid] = nblo;
     counts[tid] = tot;
     if (counts_out) counts_out[tid] = tot;
   }
@@ -98,6 +106,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const uint32_t* __restrict__
     offsets[E] = total[0];
     nb_off[E] = total[1];
     nb2_off[E] = total[2];
+    nbl_off[E] = total[3];
   }
   __syncthreads();
   if (act) {
@@ -192,7 +201,9 @@ cudaError_t launch_scan(const beam_moe_cfg& c, const Layout& L, char* ws, int32_
                                   c.n_experts, L.bn, reinterpret_cast<int32_t*>(ws + L.counts),
                                   reinterpret_cast<int32_t*>(ws + L.offsets),
                                   reinterpret_cast<int32_t*>(ws + L.nb_off),
-                                  reinterpret_cast<int32_t*>(ws + L.nb2_off), counts_out);
+                                  reinterpret_cast<int32_t*>(ws + L.nb2_off), L.light_max,
+                                  L.light_bn, reinterpret_cast<int32_t*>(ws + L.nbl_off),
+                                  counts_out);
   return cudaGetLastError();
 }
 

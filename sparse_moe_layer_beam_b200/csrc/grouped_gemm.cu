@@ -321,6 +321,22 @@ cudaError_t launch_gateup(const beam_moe_cfg& c, const Layout& L, const uint16_t
   return dispatch_bn<true>(L.bn, tw, tx, p, st);
 }
 
+cudaError_t launch_gateup_light(const beam_moe_cfg& c, const Layout& L, const uint16_t* w13,
+                                char* ws, cudaStream_t st) {
+  Layout M = L;
+  M.bn = L.light_bn;
+  M.nb_off = L.nbl_off;
+  return launch_gateup(c, M, w13, ws, st);
+}
+
+cudaError_t launch_down_light(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2,
+                              char* ws, cudaStream_t st) {
+  Layout M = L;
+  M.bn = L.light_bn;
+  M.nb_off = L.nbl_off;
+  return launch_down(c, M, w2, ws, st);
+}
+
 cudaError_t launch_down(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2, char* ws,
                         cudaStream_t st) {
   const int H = c.hidden, I = c.inter, E = c.n_experts;

@@ -21,6 +21,7 @@ constexpr int kChunkWords = kChunk / 32;
 // of one pipeline stage (64 bf16 = one 128-byte swizzle row).
 constexpr int kTileM = 128;
 constexpr int kTileK = 64;
+constexpr int kLightRows = 64;  // see Layout::light_max
 
 // Status bits written by kernels into the workspace status word.
 constexpr uint32_t kFlagProducer = 0x1;
@@ -79,11 +80,15 @@ struct Layout {
   int bn;           // token tile of the grouped GEMMs
   int pair_gateup; // 1: gate/up grouped GEMM on CTA pairs
   int pair_down;   // 1: down grouped GEMM on CTA pairs
+  int light_max;   // with CTA pairs: experts with at most this many rows go to the
+                   // one-CTA kernel instead (0: none)
+  int light_bn;    // that kernel's token tile
   size_t status;    // uint32[64]
   size_t counts;    // int32[E]
   size_t offsets;   // int32[E + 1] first row of each expert in the permuted rows
-  size_t nb_off;    // int32[E + 1] prefix of ceil(count / bn)
+  size_t nb_off;    // int32[E + 1] prefix of ceil(count / bn) (light experts: 0)
   size_t nb2_off;   // int32[E + 1] prefix of ceil(count / (2 bn))
+  size_t nbl_off;   // int32[E + 1] prefix of ceil(count / light_bn) over the light experts
   size_t ids;       // int32[T * K]
   size_t w;         // float[T * K]
   size_t pos;       // int32[T * K] permuted row of each assignment
@@ -173,6 +178,12 @@ cudaError_t launch_permute(const beam_moe_cfg& c, const Layout& L, const uint16_
                            cudaStream_t st);
 cudaError_t launch_gateup(const beam_moe_cfg& c, const Layout& L, const uint16_t* w13, char* ws,
                           cudaStream_t st);
+// The one-CTA kernels over the light experts only (L.light_max > 0), after the
+// CTA-pair kernels have done the others.
+cudaError_t launch_gateup_light(const beam_moe_cfg& c, const Layout& L, const uint16_t* w13,
+                                char* ws, cudaStream_t st);
+cudaError_t launch_down_light(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2,
+                              char* ws, cudaStream_t st);
 cudaError_t launch_down(const beam_moe_cfg& c, const Layout& L, const uint16_t* w2, char* ws,
                         cudaStream_t st);
 bool pair_gemm_supported(const beam_moe_cfg& c);

@@ -577,6 +577,7 @@ Fp4Layout make_layout_nvfp4(const beam_moe_cfg& c, int64_t T, int sms) {
   Layout& L = F.base;
   L.bn = kBN;  // token tiles of 128 rows; expert segments padded to them
   L.pair_gateup = L.pair_down = 0;
+  L.light_max = 0;
   // CTA pairs for the down GEMM once experts average 1024 rows or more. A
   // pair tile of 256 weight rows x 256 tokens halves the operand bytes per
   // FLOP, but its one 256-column accumulator leaves the MMAs idle while the

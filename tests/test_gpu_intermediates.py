@@ -210,3 +210,38 @@ def test_combine_is_the_k_ordered_fp32_sum(name, T):
     w = _read(ws, lay.w, np.float32, (wl.T, wl.K))
     y = _read(ws, lay.y, np.float32, (A, wl.H))
     assert np.array_equal(_gpu.bits_of(out), _gpu.combine_bits(y, pos, w))
+
+
+def test_light_experts_on_one_cta_tiles():
+    """With CTA pairs on (225 rows per expert on average), experts with at
+    most 64 rows run on the one-CTA kernels after the pair kernels: a
+    selection bias on three experts leaves four experts with 43 to 57 rows,
+    nine with about 180 to 215 and the three biased ones with over 550 (more
+    than their 256 weight rows: token-block-outer order). Every h element
+    against the oracle, the combine chain bit for bit, every output row
+    against the oracle."""
+    import dataclasses
+    wl = dataclasses.replace(synth.workload("tiny").with_T(900), n_hot=3, hot_bias=3.0)
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    counts = np.bincount(r["ids"].ravel(), minlength=wl.E)
+    ws, lay = _run_stages(wl, x, 4, bias=b)
+    assert lay.pair_gateup == 1 and lay.light_rows == 64
+    assert (counts <= 64).sum() >= 4 and (counts > 256).sum() >= 3
+    ids, pos = _check_dispatch(wl, x, r, ws, lay)
+    _check_h(wl, x, r, ids, pos, ws, lay, np.arange(wl.T))
+    del ws
+    cfg = _gpu.cfg_of(wl)
+    w13, w2, wrd = _gpu.device_weights(wl)
+    out = torch.empty((wl.T, wl.H), dtype=torch.int16, device="cuda")
+    ws = torch.empty(bm.beam_moe_workspace_size(cfg, wl.T), dtype=torch.uint8, device="cuda")
+    bd = torch.from_numpy(np.asarray(b, np.float32)).cuda()
+    bm.beam_moe_forward_stages(cfg, _gpu.to_dev_bits(x), wrd, bd, w13, w2, out, 6, ws)
+    assert bm.beam_moe_check(ws) == 0
+    A = wl.T * wl.K
+    y = _read(ws, lay.y, np.float32, (A, wl.H))
+    w = _read(ws, lay.w, np.float32, (wl.T, wl.K))
+    got = _gpu.bits_of(out)
+    assert np.array_equal(got, _gpu.combine_bits(y, pos, w))
+    ref = _gpu.oracle_outputs(wl, x, np.arange(wl.T), r)
+    err, _ = _gpu.max_rel_err(got, ref)
+    assert err <= _gpu.TOL
