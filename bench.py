@@ -60,11 +60,11 @@ STAGES = ("router_gemm", "router_topk", "scan", "permute", "gateup_gemm", "down_
 # chunk (2048 rows per expert in both). A record is valid only while the
 # sources of the kernel that runs hash to `sha256`; any edit voids it.
 GATEUP_TRAFFIC = {
-    "decode": {"per": "touched_expert", "bytes": 52566449,
+    "decode": {"per": "touched_expert", "bytes": 52574526,
                "sources": ("sparse_moe_layer_beam_b200/csrc/grouped_gemm.cu",
                            "sparse_moe_layer_beam_b200/csrc/grouped_gemm.cuh",
                            "sparse_moe_layer_beam_b200/csrc/sm100.cuh"),
-               "sha256": "544cfa507480c8156b1c6906677d80e9870e5cac2af85f853956469f90dced54"},
+               "sha256": "eac8298aa60b6a07f459e3937256a70250143c7d1720c3b7f80728b01fffd2d7"},
     "long": {"per": "assignment", "bytes": 96461,
              "sources": ("sparse_moe_layer_beam_b200/csrc/grouped_gemm_2sm.cu",
                          "sparse_moe_layer_beam_b200/csrc/grouped_gemm.cuh",
