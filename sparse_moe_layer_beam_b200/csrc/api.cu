@@ -61,9 +61,10 @@ Layout make_layout(const beam_moe_cfg& c, int64_t T, int sms, bool allow_tc) {
   }
   L.bn = pick_bn(T, K, E);
   // CTA pairs halve the token-row bytes each SM reads per weight byte and
-  // double-buffer the accumulator. That pays once experts average 64 rows or
-  // more (measured: prefill at 128 rows is faster on pairs for both GEMMs);
-  // below that the GEMMs stream weights and one CTA per tile is enough.
+  // double-buffer the accumulator. They run with 256-token tiles, which the
+  // tile choice above reaches once experts average more than about 102 rows
+  // (measured: prefill at 128 rows is faster on pairs for both GEMMs); below
+  // that the GEMMs stream weights and one CTA per tile is enough.
   const double mean_rows = (double)T * K / E;
   const bool pair_ok = L.bn == 256 && pair_gemm_supported(c);
   L.pair_gateup = (pair_ok && mean_rows >= 64.0) ? 1 : 0;
