@@ -200,6 +200,40 @@ def test_routed_forward_on_cta_pairs_with_dropped_and_repeated_ids():
     assert err <= _gpu.TOL
 
 
+def test_routed_forward_light_expert_bounds():
+    """Routing replay with 900 tokens (CTA pairs on): experts with exactly 64
+    rows (the largest that runs on one-CTA tiles), 65 (the smallest on pairs),
+    1 and 0 rows, the others about 290; every output row against the oracle,
+    the counts bit-exact."""
+    wl = synth.workload("tiny").with_T(900)
+    x, _, _, _, _ = _inputs.routed_inputs(wl)
+    T, K, E = wl.T, wl.K, wl.E
+    rng = np.random.default_rng(7)
+    ids = np.empty((T, K), np.int32)
+    heavy = np.arange(4, E)
+    for t in range(T):
+        first = 0 if t < 64 else 1 if t < 129 else 2 if t == 129 else None
+        rest = rng.choice(heavy, size=K if first is None else K - 1, replace=False)
+        ids[t] = rest if first is None else np.concatenate([[first], rest])
+    w = rng.uniform(0.05, 0.6, size=(T, K)).astype(np.float32)
+    counts_want = np.bincount(ids.ravel(), minlength=E)
+    assert list(counts_want[:4]) == [64, 65, 1, 0]
+    cfg = _gpu.cfg_of(wl)
+    lay = bm.beam_moe_workspace_layout(cfg, T)
+    assert lay.pair_gateup == 1 and lay.light_rows == 64
+    w13, w2, _ = _gpu.device_weights(wl)
+    out = torch.empty((T, wl.H), dtype=torch.int16, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    ws = torch.empty(bm.beam_moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    bm.beam_moe_forward_routed(cfg, _gpu.to_dev_bits(x), torch.from_numpy(ids).cuda(),
+                               torch.from_numpy(w).cuda(), w13, w2, out, ws, counts)
+    assert bm.beam_moe_check(ws) == 0
+    assert np.array_equal(counts.cpu().numpy(), counts_want)
+    ref = oracle.experts(oracle.cfg_for(wl), x, ids, w, synth.host_w13(wl), synth.host_w2(wl))
+    err, _ = _gpu.max_rel_err(_gpu.bits_of(out), ref)
+    assert err <= _gpu.TOL
+
+
 def test_route_only_entry_point():
     wl = synth.workload("decode").with_T(300)
     x, _, wr, b, r = _inputs.routed_inputs(wl)
