@@ -20,12 +20,11 @@
 // counts between route and plan, a barrier after experts). The gate/up GEMM's
 // wait for arrivals is the only place a kernel waits for another rank; it is
 // bounded (1 s, then status bit kFlagArrival). Every rank's workspace has the
-// same layout,
-// so a peer's buffer is its workspace pointer plus a fixed offset: [status]
-// [receive rows: cap x H x 4 bytes, bf16 on arrival, fp32 y after the down
-// GEMM][return addresses: cap x int32][returned y: T_max K x H fp32][h: cap x
-// I bf16][local expert counts, offsets, token-tile prefix][arrival counters: E / world
-// int32][routing scratch].
+// same layout, so a peer's buffer is its workspace pointer plus a fixed
+// offset: [status][receive rows: cap x H x 4 bytes, bf16 on arrival, fp32 y
+// after the down GEMM][return addresses: cap x int32][returned y: T_max K x H
+// fp32][h: cap x I bf16][local expert counts, offsets, token-tile prefix]
+// [arrival counters: E / world int32][routing scratch].
 #include <string.h>
 
 #include "internal.h"
