@@ -234,6 +234,25 @@ def test_routed_forward_light_expert_bounds():
     assert err <= _gpu.TOL
 
 
+@pytest.mark.parametrize("T", [300, 2000])  # one-CTA tiles of 32 tokens; CTA pairs
+def test_widest_configuration(T):
+    """The most experts and the largest top-k the library takes: 512 experts
+    in 8 groups of 64, top-4 groups, top-32 (16 experts per lane in the top-k
+    warp, 32 slots per token in the permute and the combine). Routes bit-exact,
+    every output row against the oracle."""
+    wl = synth.Workload(name="wide", T=T, H=256, I=128, E=512, G=8, Gk=4, K=32)
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    g = _gpu.forward(wl, x)
+    assert g["flags"] == 0
+    _gpu.check_routes(g, r, wl.E)
+    lay = bm.beam_moe_workspace_layout(_gpu.cfg_of(wl), T)
+    assert lay.pair_gateup == (1 if T == 2000 else 0)
+    ref = oracle.experts(oracle.cfg_for(wl), x, r["ids"], r["weights"], synth.host_w13(wl),
+                         synth.host_w2(wl))
+    err, _ = _gpu.max_rel_err(g["out"], ref)
+    assert err <= _gpu.TOL, err
+
+
 def test_route_only_entry_point():
     wl = synth.workload("decode").with_T(300)
     x, _, wr, b, r = _inputs.routed_inputs(wl)
