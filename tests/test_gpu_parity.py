@@ -253,6 +253,27 @@ def test_widest_configuration(T):
     assert err <= _gpu.TOL, err
 
 
+@pytest.mark.parametrize("E,G,Gk,K,H,T", [(4, 2, 1, 2, 128, 100),    # 2 groups of 2, keep 1
+                                           (16, 1, 1, 4, 256, 200),   # one group: no group step
+                                           (16, 4, 2, 1, 256, 150)])  # top-1: weight = scale
+def test_smallest_configurations(E, G, Gk, K, H, T):
+    """Degenerate routing shapes: the fewest experts per group the top-k warp
+    takes, a single group (the group selection keeps everything), and top-1
+    routing (renormalised, every weight is exactly the scale). Routes
+    bit-exact, every output row against the oracle."""
+    wl = synth.Workload(name="small", T=T, H=H, I=128, E=E, G=G, Gk=Gk, K=K)
+    x, _, wr, b, r = _inputs.routed_inputs(wl)
+    g = _gpu.forward(wl, x)
+    assert g["flags"] == 0
+    _gpu.check_routes(g, r, wl.E)
+    if K == 1:
+        assert np.all(g["w"] == np.float32(wl.scale))
+    ref = oracle.experts(oracle.cfg_for(wl), x, r["ids"], r["weights"], synth.host_w13(wl),
+                         synth.host_w2(wl))
+    err, _ = _gpu.max_rel_err(g["out"], ref)
+    assert err <= _gpu.TOL, err
+
+
 def test_route_only_entry_point():
     wl = synth.workload("decode").with_T(300)
     x, _, wr, b, r = _inputs.routed_inputs(wl)
