@@ -298,6 +298,7 @@ GemmParams base_params(const beam_moe_cfg& c, const Layout& L, char* ws) {
   p.E = c.n_experts;
   p.status = reinterpret_cast<unsigned*>(ws + L.status);
   p.arrive = L.arrive ? reinterpret_cast<const int32_t*>(ws + L.arrive) : nullptr;
+  p.next_tile = nullptr;  // static tile order here
   return p;
 }
 

@@ -22,6 +22,7 @@ struct GemmParams {
   unsigned* status;
   const int32_t* arrive;  // [E] or nullptr: rows arrived per expert (expert parallelism);
                           // a tile's rows are loaded once arrive[e] reaches counts[e]
+  int* next_tile;         // CTA-pair kernels: the launch's tile counter (zero at launch)
 };
 
 __host__ __device__ constexpr int pow2_at_least(int v) {

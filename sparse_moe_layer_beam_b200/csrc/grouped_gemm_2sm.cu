@@ -27,6 +27,13 @@
 // k-step beats an exact cover by several smaller boxes, and 8- to 32-row
 // boxes run slower than the 64-row box although they move fewer bytes.)
 //
+// Tiles are handed out in order at run time: the even CTA's producer takes
+// the next index from a counter in global memory and publishes it, through a
+// small ring in both CTAs' shared memory, to every role of the pair. So the
+// 74 pairs work on a window of consecutive tiles (those of one or two
+// experts) however their speeds differ, instead of drifting apart over a
+// static stride, which would spread the operands they share over more of L2.
+//
 // Roles (both CTAs have the same warps): warp 0 issues this CTA's TMA loads,
 // whose completion is counted on the even CTA's barrier; warp 1 of the even
 // CTA issues the pair's MMAs and commits to barriers in both CTAs; warps 2-5
@@ -48,6 +55,10 @@ using gg::decode_tile;
 using gg::silu_mul;
 
 constexpr int kThreads = 192;
+constexpr int kTileSlots = 8;  // tile indices in flight between the fetching producer and the rest
+// readers of each published index: the odd CTA's producer, the MMA thread and
+// the four epilogue warps of each CTA
+constexpr int kTileReaders = 1 + 1 + 2 * 4;
 constexpr int kPairM = 256;  // weight rows per pair tile
 constexpr int kPairN = 256;  // max tokens per pair tile (the token block)
 
@@ -75,7 +86,8 @@ struct PairCfg {
   static constexpr int kStages = 7;  // 225 KB of the 227 KB a CTA may use
   static constexpr int kAccCols = kPairN;  // FP32 accumulator columns per stage
   static constexpr int kTmemCols = 512;    // two accumulator stages
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+  static constexpr int kBarBytes = 512;  // mbarriers, TMEM address, abort flag, tile ring
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes;
   static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 limit");
 };
 
@@ -97,13 +109,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* tsfull = drain + 1;              // [kTileSlots] an index is in the ring
+  uint64_t* tsempty = tsfull + kTileSlots;   // [kTileSlots] every reader has it (even CTA)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tsempty + kTileSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* ring = abort_flag + 1;       // [kTileSlots] tile index, -1: no more
+  static_assert((2 * PairCfg::kStages + 5 + 2 * kTileSlots) * 8 + 8 + 4 * kTileSlots <=
+                    PairCfg::kBarBytes,
+                "barrier area");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0: the CTA that issues MMAs
   const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -115,6 +132,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[a], 2 * 128);  // epilogue threads of both CTAs
     }
     mbar_init(drain, 1);
+    for (int s = 0; s < kTileSlots; ++s) {
+      mbar_init(&tsfull[s], 1);
+      mbar_init(&tsempty[s], kTileReaders);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_w);
@@ -133,6 +154,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   // other ranks; the other roles' waits allow for that.
   const uint64_t wait_ns = p.arrive ? 3000000000ull : 1000000000ull;
   const int total = __ldg(p.nb_off + p.E) * p.n_mblk;
+  // Next tile index of this pair, in order, for every role. The even CTA's
+  // producer fetches it and publishes it to both CTAs; the others read it.
+  // -1: no tiles left; -2: a wait gave up (the role stops).
+  int tslot = 0;
+  uint32_t tphase = 0;
+  // t: the counter value taken for this slot (taken one tile ahead, so that
+  // the atomic's latency overlaps the previous tile's loads).
+  auto publish_tile = [&](int t) -> int {
+    // the readers' arrivals (some from the other CTA) come before the rewrite
+    if (!mbar_wait(&tsempty[tslot], tphase ^ 1u, abort_flag, p.status, kFlagProducer, wait_ns,
+                   true))
+      return -2;
+    const int tile = t < total ? t : -1;
+    ring[tslot] = tile;
+    st_cluster_u32(mapa_shared(smem_addr((const void*)&ring[tslot]), 1), (uint32_t)tile);
+    mbar_arrive(&tsfull[tslot]);
+    mbar_arrive_cluster(mapa_shared(smem_addr(&tsfull[tslot]), 1));
+    if (++tslot == kTileSlots) {
+      tslot = 0;
+      tphase ^= 1u;
+    }
+    return tile;
+  };
+  // Without a counter (experts with about one token block each, where tiles
+  // share no operands and the hand-out would only add latency), every role
+  // walks this pair's static stride instead.
+  const bool dynamic = p.next_tile != nullptr;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  int stile = pair;
+  auto next_static = [&]() -> int {
+    const int t = stile;
+    stile += n_pairs;
+    return t < total ? t : -1;
+  };
+  // whole_warp: all 32 lanes read (the epilogue warps; lane 0 then arrives
+  // for the warp), else one thread reads and arrives.
+  auto read_tile = [&](uint32_t flag, bool whole_warp) -> int {
+    // the index may have been stored by the other CTA, released at cluster scope
+    if (!mbar_wait(&tsfull[tslot], tphase, abort_flag, p.status, flag, wait_ns, true)) return -2;
+    const int tile = ring[tslot];
+    if (whole_warp) __syncwarp();  // every lane has read the slot
+    if (!whole_warp || lane == 0)
+      mbar_arrive_cluster(mapa_shared(smem_addr(&tsempty[tslot]), 0));
+    if (++tslot == kTileSlots) {
+      tslot = 0;
+      tphase ^= 1u;
+    }
+    return tile;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -144,7 +214,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t issued = 0;
       bool ok = true;
       int arrived_e = -1;  // the expert whose rows are known to be here
-      for (int tile = pair; tile < total && ok; tile += n_pairs) {
+      int taken = (dynamic && leader) ? atomicAdd(p.next_tile, 1) : 0;
+      for (;;) {
+        const int tile = !dynamic ? next_static()
+                         : leader ? publish_tile(taken)
+                                  : read_tile(kFlagProducer, false);
+        if (tile < 0) {
+          ok = tile == -1;
+          break;
+        }
+        if (dynamic && leader) taken = atomicAdd(p.next_tile, 1);  // used at the next tile
         int e, mb, nb;
         decode_pair_tile(tile, p, e, mb, nb);
         if (p.arrive && e != arrived_e) {
@@ -184,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             phase ^= 1u;
           }
         }
+        if (!ok) break;
       }
       // The even CTA's full barriers count both CTAs' copies: wait for the
       // last ones to land before either CTA can leave.
@@ -203,7 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = pair; tile < total && ok; tile += n_pairs) {
+      for (;;) {
+        const int tile = dynamic ? read_tile(kFlagMma, false) : next_static();
+        if (tile < 0) break;
         int e, mb, nb;
         decode_pair_tile(tile, p, e, mb, nb);
         const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
@@ -245,7 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;  // TMEM lane quadrant of this warp
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = pair; tile < total; tile += n_pairs) {
+    for (;;) {
+      const int tile = dynamic ? read_tile(kFlagEpilogue, true) : next_static();
+      if (tile < 0) break;
       int e, mb, nb;
       decode_pair_tile(tile, p, e, mb, nb);
       const int rows = min(kPairN, __ldg(p.counts + e) - nb * kPairN);
@@ -357,6 +441,10 @@ cudaError_t run_pair(const CUtensorMap& tw, const CUtensorMap& tx, const CUtenso
     return cudaSuccess;
   });
   if (err != cudaSuccess) return err;
+  if (p.next_tile) {
+    err = cudaMemsetAsync(p.next_tile, 0, sizeof(int), st);
+    if (err != cudaSuccess) return err;
+  }
   cfg.gridDim = dim3((unsigned)(2 * resident_pairs));
   return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATEUP, EPRET>, tw, tx, tx64, p, ret);
 }
@@ -377,6 +465,11 @@ GemmParams base_params(const beam_moe_cfg& c, const Layout& L, char* ws) {
   p.E = c.n_experts;
   p.status = reinterpret_cast<unsigned*>(ws + L.status);
   p.arrive = L.arrive ? reinterpret_cast<const int32_t*>(ws + L.arrive) : nullptr;
+  // Tiles handed out at run time once experts average more than one 256-token
+  // block (then an expert's tiles share operands through L2); the counter is
+  // a word of the status area past the status word itself.
+  const bool dynamic = (double)L.A > (double)kPairN * c.n_experts;
+  p.next_tile = dynamic ? reinterpret_cast<int*>(ws + L.status) + kTileCounterWord : nullptr;
   return p;
 }
 

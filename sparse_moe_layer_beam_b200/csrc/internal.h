@@ -22,6 +22,7 @@ constexpr int kChunkWords = kChunk / 32;
 constexpr int kTileM = 128;
 constexpr int kTileK = 64;
 constexpr int kLightRows = 64;  // see Layout::light_max
+constexpr int kTileCounterWord = 32;  // status-area word: the CTA-pair GEMMs' tile counter
 
 // Status bits written by kernels into the workspace status word.
 constexpr uint32_t kFlagProducer = 0x1;

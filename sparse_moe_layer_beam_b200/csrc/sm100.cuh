@@ -51,17 +51,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same with acquire semantics at cluster scope: what the other CTA wrote
+// before its release-arrive on this barrier is visible after the wait.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase of parity `parity` to complete. Gives up when
 // `*abort` is set by another role, or after `limit_ns`; then, if `abort` and
 // `status` are given, it sets `*abort`, ORs `flag` into the global status
 // word, and returns false. Both pointers may be null (drain waits at exit).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           unsigned* status, uint32_t flag,
-                                          uint64_t limit_ns = 1000000000ull) {
-  if (mbar_try_wait(bar, parity)) return true;
+                                          uint64_t limit_ns = 1000000000ull,
+                                          bool cluster_acquire = false) {
+  auto done = [&]() {
+    return cluster_acquire ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
+  if (done()) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (done()) return true;
     if ((i & 255u) == 0) {
       if (abort && *abort) return false;
       if (global_timer_ns() - t0 > limit_ns) {
@@ -238,6 +256,11 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
+}
+
+// 32-bit store to a shared::cluster address (possibly the other CTA's).
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 // Arrive on an mbarrier given by its shared::cluster address (possibly the
