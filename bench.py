@@ -65,11 +65,11 @@ GATEUP_TRAFFIC = {
                            "sparse_moe_layer_beam_b200/csrc/grouped_gemm.cuh",
                            "sparse_moe_layer_beam_b200/csrc/sm100.cuh"),
                "sha256": "725f4dd9c7269a71650243ecd4c2c23c391aabfe12ab9e3dcb7a997760ff1606"},
-    "long": {"per": "assignment", "bytes": 42525,
+    "long": {"per": "assignment", "bytes": 42326,
              "sources": ("sparse_moe_layer_beam_b200/csrc/grouped_gemm_2sm.cu",
                          "sparse_moe_layer_beam_b200/csrc/grouped_gemm.cuh",
                          "sparse_moe_layer_beam_b200/csrc/sm100.cuh"),
-             "sha256": "3b24c011b70c0f03e40fe10af4bf08f101d0a24f479ca30caea4acd00ce2d9c0"},
+             "sha256": "cebdcde26c340ca125578851fff5f185362925fc332250afcd3d3b44e9d9ac43"},
 }
 
 

@@ -155,8 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t wait_ns = p.arrive ? 3000000000ull : 1000000000ull;
   const int total = __ldg(p.nb_off + p.E) * p.n_mblk;
   // Next tile index of this pair, in order, for every role. The even CTA's
-  // producer fetches it and publishes it to both CTAs; the others read it.
-  // -1: no tiles left; -2: a wait gave up (the role stops).
+  // producer takes it from the counter and publishes it to both CTAs; the
+  // others read it. -1: no tiles left; -2: a wait gave up (the role stops).
   int tslot = 0;
   uint32_t tphase = 0;
   // t: the counter value taken for this slot (taken one tile ahead, so that
@@ -192,7 +192,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // for the warp), else one thread reads and arrives.
   auto read_tile = [&](uint32_t flag, bool whole_warp) -> int {
     // the index may have been stored by the other CTA, released at cluster scope
-    if (!mbar_wait(&tsfull[tslot], tphase, abort_flag, p.status, flag, wait_ns, true)) return -2;
+    const bool got = mbar_wait(&tsfull[tslot], tphase, abort_flag, p.status, flag, wait_ns, true);
+    // a warp leaves together, even if its lanes' waits ran out at different times
+    if (whole_warp ? !__all_sync(0xffffffffu, got) : !got) return -2;
     const int tile = ring[tslot];
     if (whole_warp) __syncwarp();  // every lane has read the slot
     if (!whole_warp || lane == 0)
